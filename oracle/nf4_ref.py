@@ -1,0 +1,198 @@
+"""Oracle for the NF4 codec: codebook, blockwise quantization, double
+quantization of the constants, dequantization to BFloat16.
+
+TEST INFRASTRUCTURE ONLY (see the package header).  numpy, float64, every
+rounding written out.
+
+What the pages fix, and the readings taken where they are silent:
+
+* "AI Glossary: QLoRA", second paragraph, and "QLoRA: Fine-Tuning 65-Billion
+  Parameter Models ...", section "1. 4-bit NormalFloat (NF4)": NF4 is a 4-bit
+  type for normally distributed values, built so that each quantization bucket
+  gets the same share of values.  The pages print no values.  Reading: the
+  levels are standard-normal quantiles at evenly spaced probabilities, taken
+  separately for the positive side (8 levels) and the negative side (7
+  levels), plus an exact zero, normalised to [-1, 1]; the outermost
+  probability is delta = 1 - (1/30 + 1/32)/2.  Parity of the numbers beyond
+  this construction: unpinned by the pages (they print none).
+* Same two passages: the frozen weights are stored as 4-bit numbers with
+  scaling constants.  Reading: absmax scaling over blocks of 64 consecutive
+  elements of the row-major flattened weight; nearest level of the scaled
+  value rounded to float32; ties to the lower index; an all-zero block gets
+  the zero level (index 7); two codes per byte, first element in the high
+  nibble.
+* "AI Glossary: QLoRA", second paragraph, and "2. Double Quantization": the
+  constants (float32) are themselves quantized.  Reading: blocks of 256
+  constants, each scaled by the block's maximum (kept in float32) and coded
+  with an unsigned linear 8-bit code k/255, nearest level, ties to the lower
+  index, code 0 when the maximum is 0.
+* "AI Glossary: QLoRA", second paragraph, and "QLoRA's Working Process":
+  the 4-bit weights are turned back into BFloat16 each time the layer is
+  used.  Reading: a' = fp32(fp32(k/255) * c1); w' = bf16(fp32(q_code * a')),
+  each product a single correctly rounded float32 multiply, bf16 by
+  round-to-nearest-even.
+"""
+
+from __future__ import annotations
+
+from statistics import NormalDist
+
+import numpy as np
+
+BLOCK = 64  # elements per absmax block
+GROUP = 256  # absmax constants per double-quantization block
+ZERO_CODE = 7  # index of the exact-zero level
+
+
+def nf4_codebook() -> np.ndarray:
+    """The 16 NF4 levels as float32, sorted ascending.
+
+    Quantile construction described in the module header ("1. 4-bit
+    NormalFloat (NF4)": equal share of values per bucket for normal data).
+    Built in float64 with the standard-library normal quantile, normalised by
+    the largest level, then rounded once to float32.
+    """
+    inv = NormalDist().inv_cdf
+    delta = 1.0 - 0.5 * (1.0 / 30.0 + 1.0 / 32.0)
+    pos_p = np.linspace(delta, 0.5, 9)[:-1]  # 8 probabilities, 0.5 excluded
+    neg_p = np.linspace(delta, 0.5, 8)[:-1]  # 7 probabilities, 0.5 excluded
+    pos = [inv(p) for p in pos_p]
+    neg = [-inv(p) for p in neg_p]
+    levels = np.array(sorted(pos + neg + [0.0]), dtype=np.float64)
+    levels = levels / levels.max()
+    return levels.astype(np.float32)
+
+
+def bf16_round(x: np.ndarray) -> np.ndarray:
+    """Round float32 values to the nearest bfloat16, ties to even.
+
+    Returns float32 values that lie on the bfloat16 grid.  Finite inputs only.
+    """
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    bits = x.view(np.uint32).astype(np.uint64)
+    lsb = (bits >> 16) & 1
+    bits = (bits + 0x7FFF + lsb) & 0xFFFF0000
+    return bits.astype(np.uint32).view(np.float32)
+
+
+def bf16_bits(x: np.ndarray) -> np.ndarray:
+    """uint16 bit patterns of float32 values that already lie on the bf16 grid."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    return (x.view(np.uint32) >> 16).astype(np.uint16)
+
+
+def _nearest_index(values: np.ndarray, levels: np.ndarray) -> np.ndarray:
+    """argmin_i |values - levels[i]| in float64, first (lowest) index on ties."""
+    d = np.abs(values.astype(np.float64)[:, None] - levels.astype(np.float64)[None, :])
+    return np.argmin(d, axis=1)
+
+
+def _level2_table() -> np.ndarray:
+    """fp32(k / 255) for k = 0..255 (the 8-bit constant code's levels)."""
+    return (np.arange(256, dtype=np.float64) / 255.0).astype(np.float32)
+
+
+def quantize_nf4(w: np.ndarray, block: int = BLOCK, group: int = GROUP):
+    """Blockwise NF4 quantization with double-quantized constants.
+
+    ``w``: any-shape array of bfloat16 values (given as float32/float64 that
+    lie on the bf16 grid), flattened row-major.
+
+    Returns ``(codes, absmax_q, absmax_scale)``:
+      codes        uint8[ceil(numel/2)]   two 4-bit codes per byte, first in
+                                          the high nibble; a missing last
+                                          element is padded with code 7
+      absmax_q     uint8[NB]              8-bit code of each block's absmax
+      absmax_scale float32[NB2]           the max absmax of each 256-group
+
+    NB = ceil(numel/64), NB2 = ceil(NB/256).  A partial last block takes its
+    absmax over the elements present; a partial last group its maximum over
+    the constants present.
+    """
+    x = np.asarray(w, dtype=np.float32).reshape(-1)
+    n = x.size
+    nb = -(-n // block)
+    q = nf4_codebook()
+
+    # Level 1: per-block absmax c_b over the elements present.
+    padded = np.zeros(nb * block, dtype=np.float32)
+    padded[:n] = x
+    present = np.zeros(nb * block, dtype=bool)
+    present[:n] = True
+    mag = np.where(present, np.abs(padded), 0.0).reshape(nb, block)
+    c = mag.max(axis=1).astype(np.float32)  # exact: a bf16 value
+
+    # Normalise: n = fp32(x / c_b) (the float64 quotient of two float32
+    # values rounded to float32 equals the correctly rounded float32 quotient).
+    cb = np.repeat(c, block)
+    with np.errstate(invalid="ignore", divide="ignore"):
+        normed = (padded.astype(np.float64) / cb.astype(np.float64)).astype(np.float32)
+    normed = np.where(cb == 0, np.float32(0.0), normed)  # all-zero block -> level 7
+    codes = _nearest_index(normed, q).astype(np.uint8)
+    codes[~present] = ZERO_CODE
+
+    # Pack two per byte: first element in the high nibble.
+    if codes.size % 2:
+        codes = np.concatenate([codes, np.array([ZERO_CODE], dtype=np.uint8)])
+    pairs = codes.reshape(-1, 2)
+    packed = ((pairs[:, 0] << 4) | pairs[:, 1]).astype(np.uint8)
+    packed = packed[: (n + 1) // 2]
+
+    # Level 2: groups of 256 constants; c1 = max; code2 = nearest k/255 to
+    # fp32(c_b / c1); code 0 when c1 == 0.
+    nb2 = -(-nb // group)
+    cpad = np.zeros(nb2 * group, dtype=np.float32)
+    cpad[:nb] = c
+    c1 = cpad.reshape(nb2, group).max(axis=1).astype(np.float32)
+    c1b = np.repeat(c1, group)[:nb]
+    with np.errstate(invalid="ignore", divide="ignore"):
+        n2 = (c.astype(np.float64) / c1b.astype(np.float64)).astype(np.float32)
+    n2 = np.where(c1b == 0, np.float32(0.0), n2)
+    code2 = _nearest_index(n2, _level2_table()).astype(np.uint8)
+    return packed, code2, c1
+
+
+def dequantize_scales(absmax_q: np.ndarray, absmax_scale: np.ndarray, group: int = GROUP) -> np.ndarray:
+    """Per-block dequantized constant a' = fp32(fp32(k/255) * c1), float32[NB]."""
+    k = np.asarray(absmax_q, dtype=np.uint8)
+    lvl = _level2_table()[k].astype(np.float64)
+    c1 = np.repeat(np.asarray(absmax_scale, dtype=np.float32), group)[: k.size].astype(np.float64)
+    return (lvl * c1).astype(np.float32)  # exact float64 product, one rounding
+
+
+def dequantize_nf4(codes: np.ndarray, absmax_q: np.ndarray, absmax_scale: np.ndarray,
+                   numel: int, block: int = BLOCK, group: int = GROUP) -> np.ndarray:
+    """Dequantize to bfloat16 values (returned as float32 on the bf16 grid).
+
+    w' = bf16(fp32(q_code * a')), a' from :func:`dequantize_scales`.
+    """
+    packed = np.asarray(codes, dtype=np.uint8)
+    nib = np.empty(packed.size * 2, dtype=np.uint8)
+    nib[0::2] = packed >> 4
+    nib[1::2] = packed & 0xF
+    nib = nib[:numel]
+    q = nf4_codebook().astype(np.float64)
+    a = dequantize_scales(absmax_q, absmax_scale, group)
+    ab = np.repeat(a, block)[:numel].astype(np.float64)
+    w32 = (q[nib] * ab).astype(np.float32)  # exact float64 product, one rounding
+    return bf16_round(w32)
+
+
+def bits_per_parameter(numel: int, block: int = BLOCK, group: int = GROUP) -> float:
+    """Stored bits per weight of the packed format (codes + both constant levels)."""
+    nb = -(-numel // block)
+    nb2 = -(-nb // group)
+    return (8.0 * ((numel + 1) // 2) + 8.0 * nb + 32.0 * nb2) / numel
+
+
+def max_half_gap() -> float:
+    """Largest distance from a value in [-1, 1] to its nearest NF4 level."""
+    q = nf4_codebook().astype(np.float64)
+    return float(np.max(np.diff(q)) / 2.0)
+
+
+__all__ = [
+    "BLOCK", "GROUP", "ZERO_CODE", "nf4_codebook", "bf16_round", "bf16_bits",
+    "quantize_nf4", "dequantize_scales", "dequantize_nf4", "bits_per_parameter",
+    "max_half_gap",
+]
