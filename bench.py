@@ -1,0 +1,343 @@
+"""Benchmark of the frozen-NF4 LoRA linear layer on B200.
+
+One step = the whole hot path on one batch: NF4 quantization of the frozen
+weight (with double-quantized constants), the forward (T = s X A and the
+fused dequant-GEMM Y = X W'^T + T B) and the backward (U, dB, the fused
+dequant-GEMM dX = dY W' + U A^T, dA), through the C ABI of libqlora.so.
+
+Workload (N = 1): the LLaMA-7B attention projection, W 4096 x 4096 bf16
+~N(0, 0.02^2) with 0.1% of entries x10, 4096 tokens, r = 64, scale 0.25,
+seeded synthetic data.  With --gpus N (torchrun, one process per GPU) every
+rank runs its own batch of 4096 tokens (weak scaling) and the adapter
+gradients dA, dB are summed over ranks with one NCCL all-reduce per step
+(the data-parallel exchange).
+
+Prints one JSON line (rank 0).  `--impl reference` times the CPU oracle (the
+float64 restatement in oracle/) on a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "QLoRA linear fwd+bwd TFLOP/s & tokens/s; small-M NF4 weight GB/s vs HBM peak"
+WORKLOAD = dict(workload="llama7b_attn_proj_qlora_linear", M=4096, K=4096, N=4096, r=64, scale=0.25,
+                outliers="0.1% x10", step="quantize_nf4 + linear_fwd + linear_bwd")
+
+
+def flops_fwd(M, K, N, r):
+    return 2 * M * N * K + 2 * M * r * (K + N)
+
+
+def flops_bwd(M, K, N, r):
+    return 2 * M * N * K + 4 * M * r * (K + N)
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return dict(hbm_gbs=float(p["hbm_gbs"]), bf16_tflops=float(p["bf16_tflops"]),
+                    bf16_tflops_sustained=float(p["bf16_tflops_sustained"]), source="measured")
+    except Exception:
+        return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = sorted(float(r[1]) for r in rows if r[1].replace(".", "").isdigit())
+        mx = max(float(r[2]) for r in rows if r[2].replace(".", "").isdigit())
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": sm[len(sm) // 2] if sm else None, "sm_max_mhz": mx, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def cpu_oracle_sample(budget_rows: int = 1024):
+    """Time the oracle on a bounded sample of the workload: quantize the whole
+    4096 x 4096 weight, then forward + backward on `budget_rows` token rows."""
+    import numpy as np
+    from bit_quantized_lora_quantize_b200 import synthetic
+    from oracle import dequantize_nf4, lora_linear_backward, lora_linear_forward, quantize_nf4
+
+    case = synthetic.attn_proj_case()
+    M, K, N, r = budget_rows, case.K, case.N, case.r
+    W = case.W.float().numpy()
+    X = case.X[:M].double().numpy()
+    dY = case.dY[:M].double().numpy()
+    A = case.A.double().numpy()
+    B = case.B.double().numpy()
+    t0 = time.perf_counter()
+    codes, aq, sc = quantize_nf4(W)
+    Wdq = dequantize_nf4(codes, aq, sc, W.size).reshape(N, K)
+    lora_linear_forward(X, Wdq, A, B, case.scale)
+    lora_linear_backward(dY, X, Wdq, A, B, case.scale)
+    dt = time.perf_counter() - t0
+    fl = flops_fwd(M, K, N, r) + flops_bwd(M, K, N, r)
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count() or 1
+    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": int(cores), "kind": "oracle",
+            "sample": f"quantize of the full 4096x4096 weight + fwd+bwd on {M} of 4096 token rows (float64 numpy)",
+            "seconds": dt, "tokens_per_s": M / dt}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    vals = []
+    for _ in range(args.warmup):
+        cpu_oracle_sample(256)
+    samples = []
+    for _ in range(args.steps):
+        s = cpu_oracle_sample(512)
+        samples.append(s)
+        vals.append(s["value"])
+    v = sorted(vals)[len(vals) // 2]
+    cb = dict(samples[-1])
+    cb["value"] = v
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": dict(WORKLOAD), "cpu_baseline": cb,
+            "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def traffic_for(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if it still
+    describes the current kernel source."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+        ent = t[kernel]
+        src = os.path.join(ROOT, "bit_quantized_lora_quantize_b200", "csrc", ent["source"])
+        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        if h != ent["source_sha256_16"]:
+            return None
+        return ent["dram_bytes_per_launch"]
+    except Exception:
+        return None
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import bit_quantized_lora_quantize_b200 as q
+    from bit_quantized_lora_quantize_b200 import build as qbuild, synthetic
+
+    qbuild.build()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    case = synthetic.attn_proj_case() if rank == 0 else synthetic.linear_case(
+        4096, 4096, 4096, 64, 0.25, 1 + 1000 * rank, outlier_frac=0.001)
+    M, K, N, r, s = case.M, case.K, case.N, case.r, case.scale
+    W = case.W.to(dev)
+    X, A, B, dY = (t.to(dev) for t in (case.X, case.A, case.B, case.dY))
+    ws = q.new_workspace(M, K, N, r, dev)
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    T = torch.empty(M, r, dtype=torch.float32, device=dev)
+    dX = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+    dA = torch.empty(K, r, dtype=torch.float32, device=dev)
+    dB = torch.empty(r, N, dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # > L2 (126 MB)
+    grads = torch.empty(K * r + r * N, dtype=torch.float32, device=dev)
+
+    def step():
+        Wp = q.qlora_quantize_nf4(W)
+        q.qlora_linear_fwd(X, Wp, A, B, s, workspace=ws, Y=Y, T_save=T)
+        q.qlora_linear_bwd(dY, X, T, Wp, A, B, s, workspace=ws, dX=dX, dA=dA, dB=dB)
+        if world > 1:
+            grads[:K * r].copy_(dA.view(-1))
+            grads[K * r:].copy_(dB.view(-1))
+            dist.all_reduce(grads)
+        return Wp
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    if q.qlora_check_status(ws) != 0:
+        raise RuntimeError("device pipeline timeout during warm-up")
+
+    # ---------------- device-resident timing (kernels only), L2 flushed between steps
+    stream = torch.cuda.current_stream()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    sampler = ClockSampler(local_rank)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    q.qlora_profile_start()
+    for i in range(args.steps):
+        flush.zero_()
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    prof = q.qlora_profile_stop()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    total_ms = sum(step_ms)
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    fl_step = flops_fwd(M, K, N, r) + flops_bwd(M, K, N, r)
+    value = fl_step * world / (ms_per_step * 1e-3) / 1e12
+    tokens_per_s = M * world / (ms_per_step * 1e-3)
+
+    # ---------------- end to end through the public API with host buffers
+    pin = lambda t: t.cpu().pin_memory()  # noqa: E731
+    hW, hX, hdY = pin(case.W), pin(case.X), pin(case.dY)
+    hdA = torch.empty(K, r, dtype=torch.float32).pin_memory()
+    hdB = torch.empty(r, N, dtype=torch.float32).pin_memory()
+    h2d = hW.numel() * 2 + hX.numel() * 2 + hdY.numel() * 2
+    d2h = hdA.numel() * 4 + hdB.numel() * 4
+
+    def e2e_step():
+        W.copy_(hW, non_blocking=True)
+        X.copy_(hX, non_blocking=True)
+        dY.copy_(hdY, non_blocking=True)
+        step()
+        hdA.copy_(dA, non_blocking=True)
+        hdB.copy_(dB, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    e2e_ms = float(t.item()) / args.steps
+    e2e_value = fl_step * world / (e2e_ms * 1e-3) / 1e12
+    if q.qlora_check_status(ws) != 0:
+        raise RuntimeError("device pipeline timeout during timing")
+
+    if rank != 0:
+        return
+    peaks = load_peaks()
+    # Dominant kernel: the fused dequant-GEMM with the larger total time.
+    fused = {k: v for k, v in prof.items() if k.startswith("fused_nf4")}
+    dom = max(fused, key=lambda k: fused[k][0])
+    dom_ms = fused[dom][0] / fused[dom][1]
+    dom_flops = 2 * M * N * K + 2 * M * r * (N if dom.endswith("fwd") else K)
+    achieved = dom_flops / (dom_ms * 1e-3) / 1e12
+    launches = sum(v[2] for v in prof.values())
+    kernels = {k: {"ms_per_call": v[0] / v[1], "calls": v[1], "share": v[0] / sum(x[0] for x in prof.values())}
+               for k, v in prof.items()}
+    cpu = cpu_oracle_sample(512) if (world == 1 and not args.no_cpu_baseline) else None
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(WORKLOAD, parallelism=f"dp{world}", global_batch_tokens=M * world,
+                       l2="flushed between timed steps (256 MB write)"),
+        "tokens_per_s": tokens_per_s,
+        "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": traffic_for(dom),
+                     "peak_source": f"{peaks['source']} bf16 burst", "ms_per_launch": dom_ms},
+        "kernels": kernels,
+        "gpu_launches": launches,
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_ms},
+        "clocks": clocks,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

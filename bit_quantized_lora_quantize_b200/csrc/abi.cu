@@ -1,0 +1,331 @@
+// C ABI of the library: argument validation, workspace layout and the
+// sequence of kernel launches for each call (declared in include/qlora.h).
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/qlora.h"
+#include "kernels.h"
+#include "nf4_host.h"
+#include "tensor_map.h"
+
+namespace qlora {
+
+namespace {
+
+thread_local std::string g_last_cuda_error;
+
+qlora_status cuda_fail(cudaError_t e) {
+  g_last_cuda_error = cudaGetErrorString(e);
+  return QLORA_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr size_t kStatusBytes = 256;
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Workspace: [status word (256 B)][T pair: bf16 M x 2rp][U pair: bf16 M x 2rp]
+//            [split partials (fp32)]
+struct WsLayout {
+  size_t t_off, u_off, part_off, total;
+};
+
+WsLayout ws_layout(int64_t M, int64_t K, int64_t N, int r) {
+  WsLayout w{};
+  const size_t pair_bytes = round_up(static_cast<size_t>(M) * 2 * lora_pad(r) * 2, 256);
+  w.t_off = kStatusBytes;
+  w.u_off = w.t_off + pair_bytes;
+  w.part_off = w.u_off + pair_bytes;
+  w.total = w.part_off + round_up(skinny_partial_bytes_max(M, K, N, r), 256);
+  return w;
+}
+
+qlora_status check_linear_shape(int64_t M, int64_t K, int64_t N, int32_t r) {
+  if (M <= 0 || K <= 0 || N <= 0 || r <= 0) return QLORA_ERR_INVALID_ARG;
+  if (M >= (int64_t(1) << 31) || K >= (int64_t(1) << 31) || N >= (int64_t(1) << 31)) return QLORA_ERR_UNSUPPORTED;
+  if (K % 64 != 0 || N % 8 != 0 || r % 8 != 0 || r > 128) return QLORA_ERR_UNSUPPORTED;
+  return QLORA_OK;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// ---------------------------------------------------------------- profiling
+// Optional per-launch timing with CUDA events recorded on the caller's
+// stream around each kernel (or kernel pair) of a call.  Off by default.
+struct ProfRec {
+  const char* name;
+  int launches;
+  cudaEvent_t a, b;
+};
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+std::vector<ProfRec> g_prof_recs;
+std::vector<cudaEvent_t> g_prof_pool;
+
+cudaEvent_t prof_event() {
+  if (!g_prof_pool.empty()) {
+    cudaEvent_t e = g_prof_pool.back();
+    g_prof_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+struct ProfScope {
+  bool on;
+  cudaStream_t st;
+  const char* name;
+  int launches;
+  cudaEvent_t a = nullptr;
+  ProfScope(cudaStream_t s, const char* n, int l) : on(false), st(s), name(n), launches(l) {
+    std::lock_guard<std::mutex> g(g_prof_mu);
+    on = g_prof_on;
+    if (on) {
+      a = prof_event();
+      cudaEventRecord(a, st);
+    }
+  }
+  void done() {
+    if (!on) return;
+    std::lock_guard<std::mutex> g(g_prof_mu);
+    cudaEvent_t b = prof_event();
+    cudaEventRecord(b, st);
+    g_prof_recs.push_back({name, launches, a, b});
+    on = false;
+  }
+};
+
+}  // namespace
+
+bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, int64_t inner, int64_t rows,
+                 int64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle swizzle) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_stride_bytes)};
+  const cuuint32_t box[2] = {box_inner, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace qlora
+
+using namespace qlora;
+
+extern "C" {
+
+qlora_status qlora_quantize_nf4(const uint16_t* W, int64_t numel, uint8_t* codes, uint8_t* absmax_q,
+                                float* absmax_scale, void* stream) {
+  if (!W || !codes || !absmax_q || !absmax_scale || numel <= 0) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(codes) || (reinterpret_cast<uintptr_t>(absmax_scale) & 3u))
+    return QLORA_ERR_ALIGNMENT;
+  if (numel > (int64_t(1) << 46)) return QLORA_ERR_UNSUPPORTED;
+  ProfScope p(static_cast<cudaStream_t>(stream), "quantize_nf4", 1);
+  const cudaError_t e = launch_quantize_nf4(W, numel, codes, absmax_q, absmax_scale, nf4_params(),
+                                            static_cast<cudaStream_t>(stream));
+  p.done();
+  return e == cudaSuccess ? QLORA_OK : cuda_fail(e);
+}
+
+qlora_status qlora_dequantize_nf4(const uint8_t* codes, const uint8_t* absmax_q, const float* absmax_scale,
+                                  int64_t numel, uint16_t* W_out, void* stream) {
+  if (!codes || !absmax_q || !absmax_scale || !W_out || numel <= 0) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(codes) || !aligned16(W_out) || (reinterpret_cast<uintptr_t>(absmax_scale) & 3u))
+    return QLORA_ERR_ALIGNMENT;
+  if (numel > (int64_t(1) << 46)) return QLORA_ERR_UNSUPPORTED;
+  ProfScope p(static_cast<cudaStream_t>(stream), "dequantize_nf4", 1);
+  const cudaError_t e = launch_dequantize_nf4(codes, absmax_q, absmax_scale, numel, W_out, nf4_params(),
+                                              static_cast<cudaStream_t>(stream));
+  p.done();
+  return e == cudaSuccess ? QLORA_OK : cuda_fail(e);
+}
+
+size_t qlora_workspace_bytes(int64_t M, int64_t K, int64_t N, int32_t r) {
+  if (check_linear_shape(M, K, N, r) != QLORA_OK) return 0;
+  return ws_layout(M, K, N, r).total;
+}
+
+qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, int64_t K, int64_t N, const uint8_t* codes,
+                              const uint8_t* absmax_q, const float* absmax_scale, const uint16_t* A,
+                              const uint16_t* B, int32_t r, float scale, uint16_t* Y, float* T_save,
+                              void* workspace, size_t ws_bytes, void* stream) {
+  if (!X || !codes || !absmax_q || !absmax_scale || !A || !B || !Y || !T_save) return QLORA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return QLORA_ERR_INVALID_ARG;
+  const qlora_status sh = check_linear_shape(M, K, N, r);
+  if (sh != QLORA_OK) return sh;
+  if (!aligned16(X) || !aligned16(codes) || !aligned16(A) || !aligned16(B) || !aligned16(Y) || !aligned16(T_save) ||
+      (reinterpret_cast<uintptr_t>(absmax_scale) & 3u))
+    return QLORA_ERR_ALIGNMENT;
+  const WsLayout wl = ws_layout(M, K, N, r);
+  if (!workspace || ws_bytes < wl.total) return QLORA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return QLORA_ERR_ALIGNMENT;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int* status = reinterpret_cast<int*>(ws);
+  float* partial = reinterpret_cast<float*>(ws + wl.part_off);
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Nf4Params& P = nf4_params();
+
+  uint16_t* Tpair = reinterpret_cast<uint16_t*>(ws + wl.t_off);
+
+  ProfScope p1(st, "lora_down_xa", 2);
+  cudaError_t e = launch_skinny(SkinnyKind::kXA, X, A, M, K, N, r, scale, SkinnyOut{T_save, Tpair}, partial, status, st);
+  p1.done();
+  if (e != cudaSuccess) return cuda_fail(e);
+  ProfScope p2(st, "fused_nf4_fwd", 1);
+  e = launch_fused_fwd(X, codes, absmax_q, absmax_scale, Tpair, B, M, K, N, r, Y, status, P, st);
+  p2.done();
+  if (e != cudaSuccess) return cuda_fail(e);
+  return QLORA_OK;
+}
+
+qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float* T_save, int64_t M, int64_t K,
+                              int64_t N, const uint8_t* codes, const uint8_t* absmax_q, const float* absmax_scale,
+                              const uint16_t* A, const uint16_t* B, int32_t r, float scale, uint16_t* dX, float* dA,
+                              float* dB, void* workspace, size_t ws_bytes, void* stream) {
+  if (!dY || !X || !T_save || !codes || !absmax_q || !absmax_scale || !A || !B || !dX || !dA || !dB)
+    return QLORA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return QLORA_ERR_INVALID_ARG;
+  const qlora_status sh = check_linear_shape(M, K, N, r);
+  if (sh != QLORA_OK) return sh;
+  if (!aligned16(dY) || !aligned16(X) || !aligned16(T_save) || !aligned16(codes) || !aligned16(A) ||
+      !aligned16(B) || !aligned16(dX) || !aligned16(dA) || !aligned16(dB) ||
+      (reinterpret_cast<uintptr_t>(absmax_scale) & 3u))
+    return QLORA_ERR_ALIGNMENT;
+  const WsLayout wl = ws_layout(M, K, N, r);
+  if (!workspace || ws_bytes < wl.total) return QLORA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return QLORA_ERR_ALIGNMENT;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int* status = reinterpret_cast<int*>(ws);
+  uint16_t* Tpair = reinterpret_cast<uint16_t*>(ws + wl.t_off);
+  uint16_t* Upair = reinterpret_cast<uint16_t*>(ws + wl.u_off);
+  float* partial = reinterpret_cast<float*>(ws + wl.part_off);
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Nf4Params& P = nf4_params();
+
+  ProfScope p1(st, "lora_u_dybt", 2);
+  cudaError_t e = launch_skinny(SkinnyKind::kDyBt, dY, B, M, K, N, r, scale, SkinnyOut{nullptr, Upair}, partial,
+                                status, st);
+  p1.done();
+  if (e != cudaSuccess) return cuda_fail(e);
+  ProfScope p2(st, "lora_db_ttdy", 3);
+  e = launch_split_pair(T_save, M, r, Tpair, st);
+  if (e == cudaSuccess)
+    e = launch_skinny(SkinnyKind::kTtDy, dY, Tpair, M, K, N, r, 1.0f, SkinnyOut{dB, nullptr}, partial, status, st);
+  p2.done();
+  if (e != cudaSuccess) return cuda_fail(e);
+  ProfScope p3(st, "fused_nf4_dx", 1);
+  e = launch_fused_dx(dY, codes, absmax_q, absmax_scale, Upair, A, M, K, N, r, dX, status, P, st);
+  p3.done();
+  if (e != cudaSuccess) return cuda_fail(e);
+  ProfScope p4(st, "lora_da_xtu", 2);
+  e = launch_skinny(SkinnyKind::kXtU, X, Upair, M, K, N, r, 1.0f, SkinnyOut{dA, nullptr}, partial, status, st);
+  p4.done();
+  if (e != cudaSuccess) return cuda_fail(e);
+  return QLORA_OK;
+}
+
+qlora_status qlora_check_status(void* workspace, void* stream) {
+  if (!workspace) return QLORA_ERR_INVALID_ARG;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  int word = 0;
+  e = cudaMemcpy(&word, workspace, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (word == 0) return QLORA_OK;
+  const int zero = 0;
+  e = cudaMemcpy(workspace, &zero, sizeof(int), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return QLORA_ERR_TIMEOUT;
+}
+
+void qlora_nf4_codebook(float out[16]) {
+  if (!out) return;
+  const Nf4Params& P = nf4_params();
+  std::memcpy(out, P.q, sizeof(P.q));
+}
+
+const char* qlora_status_string(qlora_status s) {
+  switch (s) {
+    case QLORA_OK: return "ok";
+    case QLORA_ERR_INVALID_ARG: return "invalid argument";
+    case QLORA_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case QLORA_ERR_UNSUPPORTED: return "unsupported shape";
+    case QLORA_ERR_WORKSPACE: return "workspace missing or too small";
+    case QLORA_ERR_CUDA: return "CUDA error";
+    case QLORA_ERR_TIMEOUT: return "kernel pipeline wait timed out";
+  }
+  return "unknown status";
+}
+
+const char* qlora_last_cuda_error(void) { return g_last_cuda_error.c_str(); }
+
+void qlora_profile_start(void) {
+  std::lock_guard<std::mutex> g(g_prof_mu);
+  for (auto& r : g_prof_recs) {
+    g_prof_pool.push_back(r.a);
+    g_prof_pool.push_back(r.b);
+  }
+  g_prof_recs.clear();
+  g_prof_on = true;
+}
+
+int qlora_profile_stop(int max_entries, char* names, float* total_ms, int* calls, int* launches) {
+  std::lock_guard<std::mutex> g(g_prof_mu);
+  g_prof_on = false;
+  std::map<std::string, std::pair<double, std::pair<int, int>>> agg;
+  for (auto& r : g_prof_recs) {
+    float ms = 0.0f;
+    if (cudaEventSynchronize(r.b) == cudaSuccess && cudaEventElapsedTime(&ms, r.a, r.b) == cudaSuccess) {
+      auto& e = agg[r.name];
+      e.first += ms;
+      e.second.first += 1;
+      e.second.second += r.launches;
+    }
+    g_prof_pool.push_back(r.a);
+    g_prof_pool.push_back(r.b);
+  }
+  g_prof_recs.clear();
+  int n = 0;
+  for (auto& kv : agg) {
+    if (n >= max_entries) break;
+    if (names) {
+      std::strncpy(names + 48 * n, kv.first.c_str(), 47);
+      names[48 * n + 47] = 0;
+    }
+    if (total_ms) total_ms[n] = static_cast<float>(kv.second.first);
+    if (calls) calls[n] = kv.second.second.first;
+    if (launches) launches[n] = kv.second.second.second;
+    ++n;
+  }
+  return n;
+}
+
+}  // extern "C"

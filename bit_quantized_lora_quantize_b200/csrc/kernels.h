@@ -1,0 +1,65 @@
+// Internal host-side launch interface between the C-ABI layer (abi.cu) and
+// the kernels.  Not part of the public header.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "nf4_device.cuh"
+
+namespace qlora {
+
+cudaError_t launch_quantize_nf4(const uint16_t* W, int64_t numel, uint8_t* codes, uint8_t* absmax_q,
+                                float* absmax_scale, const Nf4Params& P, cudaStream_t stream);
+
+cudaError_t launch_dequantize_nf4(const uint8_t* codes, const uint8_t* absmax_q, const float* absmax_scale,
+                                  int64_t numel, uint16_t* out, const Nf4Params& P, cudaStream_t stream);
+
+// The rank-r intermediates T = s X A and U = s dY B^T enter the tensor-core
+// products as a bf16 pair matrix [rows x 2*rp] (rp = r rounded up to 64):
+// columns [0, r) hold hi = bf16(v), columns [rp, rp + r) hold
+// lo = bf16(v - hi), all other columns are 0.  hi + lo carries v to about 16
+// significant bits, so rounding the intermediates costs no accuracy.
+inline int lora_pad(int r) { return (r + 63) / 64 * 64; }
+
+// Fused dequant-GEMM, forward: Y[M,N] = X[M,K] W'[N,K]^T + (T_hi + T_lo)[M,r] B[r,N].
+cudaError_t launch_fused_fwd(const uint16_t* X, const uint8_t* codes, const uint8_t* absmax_q,
+                             const float* absmax_scale, const uint16_t* Tpair, const uint16_t* B, int64_t M, int64_t K,
+                             int64_t N, int r, uint16_t* Y, int* status, const Nf4Params& P, cudaStream_t stream);
+
+// Fused dequant-GEMM, input gradient: dX[M,K] = dY[M,N] W'[N,K] + (U_hi + U_lo)[M,r] A[K,r]^T.
+cudaError_t launch_fused_dx(const uint16_t* dY, const uint8_t* codes, const uint8_t* absmax_q,
+                            const float* absmax_scale, const uint16_t* Upair, const uint16_t* A, int64_t M, int64_t K,
+                            int64_t N, int r, uint16_t* dX, int* status, const Nf4Params& P, cudaStream_t stream);
+
+// Skinny rank-r products (split over the reduction, deterministic reduction):
+//   kXA   T  = s * X A          [M, r]   -> f32 (may be null) and pair
+//   kDyBt U  = s * dY B^T       [M, r]   -> f32 (may be null) and pair
+//   kTtDy dB = T^T dY  (fp32)   [r, N]   P1 = T pair
+//   kXtU  dA = X^T U   (fp32)   [K, r]   P1 = U pair
+enum class SkinnyKind { kXA, kDyBt, kTtDy, kXtU };
+
+struct SkinnyPlan {
+  int tiles;        // 128-row output tiles
+  int splits;       // reduction splits
+  int kb_per_split; // 64-wide reduction blocks per split
+  int bn;           // output columns of the product (rp or 2*rp)
+  size_t partial_bytes;
+};
+
+struct SkinnyOut {
+  float* f32;
+  uint16_t* pair;
+};
+
+SkinnyPlan plan_skinny(SkinnyKind kind, int64_t M, int64_t K, int64_t N, int r);
+
+cudaError_t launch_skinny(SkinnyKind kind, const uint16_t* P0, const uint16_t* P1, int64_t M, int64_t K, int64_t N,
+                          int r, float scale, SkinnyOut out, float* partial, int* status, cudaStream_t stream);
+
+// Pair matrix of a float32 [rows x r] matrix.
+cudaError_t launch_split_pair(const float* v, int64_t rows, int r, uint16_t* pair, cudaStream_t stream);
+
+size_t skinny_partial_bytes_max(int64_t M, int64_t K, int64_t N, int r);
+
+}  // namespace qlora

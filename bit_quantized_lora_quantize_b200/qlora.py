@@ -1,0 +1,227 @@
+"""Thin Python binding of ``libqlora.so`` (C ABI declared in include/qlora.h).
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels.  PyTorch supplies device memory and the current stream.  There is no
+CPU fallback: if the library is missing or the device is not a CUDA device,
+the calls raise.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libqlora.so")
+
+QLORA_OK = 0
+STATUS_NAMES = {0: "QLORA_OK", 1: "QLORA_ERR_INVALID_ARG", 2: "QLORA_ERR_ALIGNMENT", 3: "QLORA_ERR_UNSUPPORTED",
+                4: "QLORA_ERR_WORKSPACE", 5: "QLORA_ERR_CUDA", 6: "QLORA_ERR_TIMEOUT"}
+
+# Exported symbols and their C signatures.
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_SIGS = {
+    "qlora_quantize_nf4": (ctypes.c_int, [_P, _I64, _P, _P, _P, _P]),
+    "qlora_dequantize_nf4": (ctypes.c_int, [_P, _P, _P, _I64, _P, _P]),
+    "qlora_linear_fwd": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, ctypes.c_int32, ctypes.c_float,
+                                        _P, _P, _P, ctypes.c_size_t, _P]),
+    "qlora_linear_bwd": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P, _P, ctypes.c_int32,
+                                        ctypes.c_float, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "qlora_workspace_bytes": (ctypes.c_size_t, [_I64, _I64, _I64, ctypes.c_int32]),
+    "qlora_check_status": (ctypes.c_int, [_P, _P]),
+    "qlora_nf4_codebook": (None, [ctypes.POINTER(ctypes.c_float)]),
+    "qlora_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "qlora_last_cuda_error": (ctypes.c_char_p, []),
+    "qlora_profile_start": (None, []),
+    "qlora_profile_stop": (ctypes.c_int, [ctypes.c_int, ctypes.c_char_p, ctypes.POINTER(ctypes.c_float),
+                                          ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]),
+}
+
+_lib = None
+
+
+class QloraError(RuntimeError):
+    def __init__(self, fn: str, status: int, detail: str = ""):
+        self.status = status
+        msg = f"{fn} -> {STATUS_NAMES.get(status, status)}"
+        if detail:
+            msg += f" ({detail})"
+        super().__init__(msg)
+
+
+def lib() -> ctypes.CDLL:
+    """Load libqlora.so (built in-tree by ``build.py``); raise if absent."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"CUDA library not built: {LIB_PATH} is missing (run bit_quantized_lora_quantize_b200/build.py)")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            f = getattr(handle, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def _check(fn: str, status: int) -> None:
+    if status != QLORA_OK:
+        detail = ""
+        if status == 5:
+            detail = lib().qlora_last_cuda_error().decode()
+        raise QloraError(fn, status, detail)
+
+
+def _ptr(t: torch.Tensor) -> int:
+    return t.data_ptr()
+
+
+def _require_cuda(*ts: torch.Tensor) -> None:
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError("qlora kernels take CUDA tensors only (no CPU path)")
+        if not t.is_contiguous():
+            raise ValueError("qlora kernels take contiguous tensors")
+
+
+def _stream() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+# ---------------------------------------------------------------- packed weight
+@dataclass
+class PackedNF4:
+    """A frozen weight [N, K] in the packed NF4 format of include/qlora.h."""
+
+    codes: torch.Tensor         # uint8 [ceil(N*K/2)]
+    absmax_q: torch.Tensor      # uint8 [NB]
+    absmax_scale: torch.Tensor  # float32 [NB2]
+    shape: tuple
+
+    @property
+    def numel(self) -> int:
+        n = 1
+        for s in self.shape:
+            n *= s
+        return n
+
+
+def packed_sizes(numel: int):
+    nb = -(-numel // 64)
+    return (numel + 1) // 2, nb, -(-nb // 256)
+
+
+def qlora_nf4_codebook() -> list:
+    buf = (ctypes.c_float * 16)()
+    lib().qlora_nf4_codebook(buf)
+    return list(buf)
+
+
+def qlora_quantize_nf4(W: torch.Tensor) -> PackedNF4:
+    """Quantize a bf16 CUDA tensor (any shape, flattened row-major)."""
+    _require_cuda(W)
+    if W.dtype != torch.bfloat16:
+        raise ValueError("W must be bfloat16")
+    n = W.numel()
+    nc, nb, nb2 = packed_sizes(n)
+    dev = W.device
+    codes = torch.empty(max(nc, 16), dtype=torch.uint8, device=dev)[:nc]
+    aq = torch.empty(nb, dtype=torch.uint8, device=dev)
+    sc = torch.empty(nb2, dtype=torch.float32, device=dev)
+    _check("qlora_quantize_nf4", lib().qlora_quantize_nf4(_ptr(W), n, _ptr(codes), _ptr(aq), _ptr(sc), _stream()))
+    return PackedNF4(codes, aq, sc, tuple(W.shape))
+
+
+def qlora_dequantize_nf4(p: PackedNF4) -> torch.Tensor:
+    _require_cuda(p.codes, p.absmax_q, p.absmax_scale)
+    out = torch.empty(p.shape, dtype=torch.bfloat16, device=p.codes.device)
+    _check("qlora_dequantize_nf4", lib().qlora_dequantize_nf4(_ptr(p.codes), _ptr(p.absmax_q), _ptr(p.absmax_scale),
+                                                              p.numel, _ptr(out), _stream()))
+    return out
+
+
+def qlora_workspace_bytes(M: int, K: int, N: int, r: int) -> int:
+    return int(lib().qlora_workspace_bytes(M, K, N, r))
+
+
+def new_workspace(M: int, K: int, N: int, r: int, device) -> torch.Tensor:
+    nbytes = qlora_workspace_bytes(M, K, N, r)
+    if nbytes == 0:
+        raise QloraError("qlora_workspace_bytes", 3, f"M={M} K={K} N={N} r={r}")
+    return torch.zeros(nbytes, dtype=torch.uint8, device=device)
+
+
+def qlora_linear_fwd(X: torch.Tensor, W: PackedNF4, A: torch.Tensor, B: torch.Tensor, scale: float,
+                     workspace: torch.Tensor | None = None, Y: torch.Tensor | None = None,
+                     T_save: torch.Tensor | None = None):
+    """Return (Y, T_save) for Y = X W'^T + (s X A) B (see include/qlora.h)."""
+    M, K = X.shape
+    N = W.shape[0]
+    r = A.shape[1]
+    _require_cuda(X, A, B, W.codes)
+    dev = X.device
+    if workspace is None:
+        workspace = new_workspace(M, K, N, r, dev)
+    if Y is None:
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    if T_save is None:
+        T_save = torch.empty(M, r, dtype=torch.float32, device=dev)
+    _check("qlora_linear_fwd", lib().qlora_linear_fwd(
+        _ptr(X), M, K, N, _ptr(W.codes), _ptr(W.absmax_q), _ptr(W.absmax_scale), _ptr(A), _ptr(B), r,
+        float(scale), _ptr(Y), _ptr(T_save), _ptr(workspace), workspace.numel(), _stream()))
+    return Y, T_save
+
+
+def qlora_linear_bwd(dY: torch.Tensor, X: torch.Tensor, T_save: torch.Tensor, W: PackedNF4, A: torch.Tensor,
+                     B: torch.Tensor, scale: float, workspace: torch.Tensor | None = None,
+                     dX: torch.Tensor | None = None, dA: torch.Tensor | None = None, dB: torch.Tensor | None = None):
+    """Return (dX, dA, dB) (see include/qlora.h)."""
+    M, K = X.shape
+    N = W.shape[0]
+    r = A.shape[1]
+    _require_cuda(dY, X, T_save, A, B, W.codes)
+    dev = X.device
+    if workspace is None:
+        workspace = new_workspace(M, K, N, r, dev)
+    if dX is None:
+        dX = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+    if dA is None:
+        dA = torch.empty(K, r, dtype=torch.float32, device=dev)
+    if dB is None:
+        dB = torch.empty(r, N, dtype=torch.float32, device=dev)
+    _check("qlora_linear_bwd", lib().qlora_linear_bwd(
+        _ptr(dY), _ptr(X), _ptr(T_save), M, K, N, _ptr(W.codes), _ptr(W.absmax_q), _ptr(W.absmax_scale), _ptr(A),
+        _ptr(B), r, float(scale), _ptr(dX), _ptr(dA), _ptr(dB), _ptr(workspace), workspace.numel(), _stream()))
+    return dX, dA, dB
+
+
+def qlora_check_status(workspace: torch.Tensor) -> int:
+    """Synchronise and return the device status code (0 = OK, 6 = a pipeline wait timed out)."""
+    return int(lib().qlora_check_status(_ptr(workspace), _stream()))
+
+
+def qlora_profile_start() -> None:
+    lib().qlora_profile_start()
+
+
+def qlora_profile_stop(max_entries: int = 32) -> dict:
+    """Per-kernel {name: (total_ms, records, launches)} since qlora_profile_start."""
+    names = ctypes.create_string_buffer(48 * max_entries)
+    ms = (ctypes.c_float * max_entries)()
+    calls = (ctypes.c_int * max_entries)()
+    launches = (ctypes.c_int * max_entries)()
+    n = lib().qlora_profile_stop(max_entries, names, ms, calls, launches)
+    out = {}
+    for i in range(n):
+        name = names.raw[48 * i:48 * (i + 1)].split(b"\0", 1)[0].decode()
+        out[name] = (float(ms[i]), int(calls[i]), int(launches[i]))
+    return out
+
+
+__all__ = ["qlora_profile_start", "qlora_profile_stop", "LIB_PATH", "lib", "QloraError", "PackedNF4", "packed_sizes", "qlora_nf4_codebook", "qlora_quantize_nf4",
+           "qlora_dequantize_nf4", "qlora_workspace_bytes", "new_workspace", "qlora_linear_fwd", "qlora_linear_bwd",
+           "qlora_check_status"]

@@ -1,0 +1,187 @@
+/*
+ * qlora.h -- C ABI of the frozen-NF4 linear layer with a LoRA adapter,
+ * for NVIDIA B200 (sm_100a).
+ *
+ * What the calls compute (sources are the web pages on QLoRA this library
+ * restates; they describe the method in prose, without formulas):
+ *   - "AI Glossary: QLoRA" (mangrove.ai), definition and second paragraph:
+ *     the frozen weights are stored as 4-bit numbers; each time the layer is
+ *     used they are turned back into BFloat16 for the product; weight
+ *     gradients are computed only for the LoRA matrices; NF4 is the 4-bit
+ *     type for normally distributed values; the scaling constants are
+ *     themselves quantized.
+ *   - "QLoRA: Fine-Tuning 65-Billion Parameter Models on a Single Consumer
+ *     GPU" (deepfa.ir): "LoRA: Prerequisite for Understanding QLoRA" (the
+ *     update is a d x r times r x k product), "QLoRA's Technical Innovations"
+ *     (1. 4-bit NormalFloat, 2. Double Quantization) and "QLoRA's Working
+ *     Process" (quantize, freeze, add bf16 adapters, backpropagate through the
+ *     frozen 4-bit weights, dequantize on the fly).
+ *
+ * Conventions shared by every call:
+ *   - bf16 tensors are passed as uint16_t bit patterns; all tensors are
+ *     row-major and contiguous.
+ *   - W  [N x K]  frozen weight (out x in).  X [M x K].  A [K x r].
+ *     B [r x N].  Y, dY [M x N].  The LoRA scale s is a float argument.
+ *   - Every pointer is a DEVICE pointer, 16-byte aligned, allocated and owned
+ *     by the caller.  The library allocates no device memory and frees none.
+ *   - `stream` is a cudaStream_t (passed as void*); every call only enqueues
+ *     work on it and returns without synchronising.
+ *   - Arguments are validated on the host before anything is launched; an
+ *     invalid call returns an error and enqueues nothing.  QLORA_ERR_CUDA
+ *     means a launch failed (see qlora_last_cuda_error).
+ *
+ * Packed NF4 format (the layout every call below agrees on):
+ *   - Flatten W row-major; blocks of 64 consecutive elements share one
+ *     absmax constant c_b; groups of 256 consecutive blocks share one float
+ *     c1 = max c_b.  NB = ceil(numel / 64) blocks, NB2 = ceil(NB / 256) groups.
+ *   - codes        uint8[ceil(numel / 2)]: element 2j in the high nibble of
+ *                  byte j, element 2j + 1 in the low nibble; the code is the
+ *                  index (0..15) of the nearest NF4 level to fp32(x / c_b),
+ *                  ties to the lower index, 7 (the exact zero) for an
+ *                  all-zero block and for a padding nibble.
+ *   - absmax_q     uint8[NB]: nearest k in 0..255 of fp32(k / 255) to
+ *                  fp32(c_b / c1), ties to the lower k, 0 when c1 = 0.
+ *   - absmax_scale float[NB2]: c1 per group.
+ *   - Dequantized weight: a' = fp32(fp32(k / 255) * c1),
+ *                         w' = bf16_rne(fp32(q[code] * a')).
+ */
+#ifndef QLORA_H
+#define QLORA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define QLORA_API __attribute__((visibility("default")))
+#else
+#define QLORA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  QLORA_OK = 0,
+  QLORA_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, non-finite scale */
+  QLORA_ERR_ALIGNMENT = 2,   /* a pointer is not 16-byte aligned */
+  QLORA_ERR_UNSUPPORTED = 3, /* a shape outside the supported set (see each call) */
+  QLORA_ERR_WORKSPACE = 4,   /* workspace pointer null or smaller than qlora_workspace_bytes */
+  QLORA_ERR_CUDA = 5,        /* a CUDA launch or query failed */
+  QLORA_ERR_TIMEOUT = 6      /* a kernel gave up waiting on a pipeline barrier (qlora_check_status) */
+} qlora_status;
+
+/*
+ * Blockwise NF4 quantization with double-quantized constants.
+ * "AI Glossary: QLoRA", second paragraph; "1. 4-bit NormalFloat (NF4)" and
+ * "2. Double Quantization" in "QLoRA: Fine-Tuning 65-Billion Parameter
+ * Models ...".
+ *   W             in   bf16[numel]      any numel >= 1 (a partial last block
+ *                                       takes its absmax over the elements
+ *                                       present, a partial last group its max
+ *                                       over the constants present)
+ *   codes         out  uint8[ceil(numel/2)]
+ *   absmax_q      out  uint8[NB]
+ *   absmax_scale  out  float[NB2]
+ * Deterministic: the result depends only on W.
+ */
+QLORA_API qlora_status qlora_quantize_nf4(const uint16_t* W, int64_t numel, uint8_t* codes, uint8_t* absmax_q,
+                                float* absmax_scale, void* stream);
+
+/*
+ * Dequantization to bf16 (the weight the linear calls multiply by).
+ * "AI Glossary: QLoRA", second paragraph (4-bit weights turned back into
+ * BFloat16 for the calculation).
+ *   codes, absmax_q, absmax_scale  in   packed format above, for numel weights
+ *   W_out                          out  bf16[numel]
+ */
+QLORA_API qlora_status qlora_dequantize_nf4(const uint8_t* codes, const uint8_t* absmax_q, const float* absmax_scale,
+                                  int64_t numel, uint16_t* W_out, void* stream);
+
+/*
+ * Forward of the frozen-NF4 linear layer with a LoRA adapter.
+ * "AI Glossary: QLoRA", second paragraph; "LoRA: Prerequisite for
+ * Understanding QLoRA"; "QLoRA's Working Process", steps 3-4.
+ *   T_save = fp32(s * X A)                [M x r]   (kept for the backward)
+ *   Y      = bf16(X W'^T + T_save B)      [M x N]   (fp32 accumulation)
+ * where W' is the dequantized weight, decoded tile by tile inside the
+ * product (no bf16 copy of W is written).  T enters the tensor-core product
+ * as the bf16 pair hi = bf16(T), lo = bf16(T - hi) (about 16 significant
+ * bits), so it loses no accuracy to a bf16 rounding.
+ *   X             in   bf16[M x K]
+ *   codes...      in   packed W [N x K] (numel = N*K)
+ *   A             in   bf16[K x r]
+ *   B             in   bf16[r x N]
+ *   Y             out  bf16[M x N]
+ *   T_save        out  float[M x r]
+ *   workspace     in/out device scratch of at least qlora_workspace_bytes(M,K,N,r)
+ *                 bytes; contents on entry are ignored, except that the
+ *                 first 256 bytes hold the status word read by
+ *                 qlora_check_status (clear them once with zeros).
+ * Supported: K % 64 == 0, N % 8 == 0, r % 8 == 0 with 8 <= r <= 128,
+ * M, N, K < 2^31.  Otherwise QLORA_ERR_UNSUPPORTED.
+ */
+QLORA_API qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, int64_t K, int64_t N, const uint8_t* codes,
+                              const uint8_t* absmax_q, const float* absmax_scale, const uint16_t* A,
+                              const uint16_t* B, int32_t r, float scale, uint16_t* Y, float* T_save,
+                              void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Backward of the same layer for an upstream gradient dY.  Gradients are
+ * produced only for the adapter; the frozen base weight gets none
+ * ("AI Glossary: QLoRA", second paragraph; "QLoRA's Working Process",
+ * step 5: gradients flow through the frozen 4-bit weights into LoRA).
+ *   U  = s * dY B^T           fp32        [M x r]   (workspace, as a bf16 pair)
+ *   dB = T_save^T dY          fp32        [r x N]
+ *   dX = bf16(dY W' + U A^T)              [M x K]
+ *   dA = X^T U                fp32        [K x r]
+ *   dY, X          in   bf16
+ *   T_save         in   float[M x r] as written by qlora_linear_fwd
+ *   dX             out  bf16[M x K]
+ *   dA, dB         out  float (overwritten, not accumulated)
+ * Same supported shapes and workspace rule as qlora_linear_fwd.  The
+ * reductions over M are split across thread blocks and summed in a fixed
+ * order: results are bit-reproducible run to run.
+ */
+QLORA_API qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float* T_save, int64_t M, int64_t K,
+                              int64_t N, const uint8_t* codes, const uint8_t* absmax_q, const float* absmax_scale,
+                              const uint16_t* A, const uint16_t* B, int32_t r, float scale, uint16_t* dX, float* dA,
+                              float* dB, void* workspace, size_t ws_bytes, void* stream);
+
+/* Workspace bytes needed by qlora_linear_fwd / qlora_linear_bwd for these sizes
+ * (0 for an unsupported shape). */
+QLORA_API size_t qlora_workspace_bytes(int64_t M, int64_t K, int64_t N, int32_t r);
+
+/* Synchronises `stream`, then reads the status word at the start of
+ * `workspace`: QLORA_OK, or QLORA_ERR_TIMEOUT if a kernel of an earlier call
+ * gave up on a pipeline wait (its outputs are then undefined).  The word is
+ * reset to zero. */
+QLORA_API qlora_status qlora_check_status(void* workspace, void* stream);
+
+/* The 16 NF4 levels (float32, ascending) this library encodes against. */
+QLORA_API void qlora_nf4_codebook(float out[16]);
+
+/* Static description of a status code. */
+QLORA_API const char* qlora_status_string(qlora_status s);
+
+/* The last CUDA error string seen by a call of this thread ("" if none). */
+QLORA_API const char* qlora_last_cuda_error(void);
+
+/*
+ * Optional kernel timing (no counterpart on the pages; measurement support).
+ * qlora_profile_start clears earlier records and makes every later call of
+ * this library record a pair of CUDA events on its stream around each of its
+ * kernels (the rank-r products count their split and reduction launches as
+ * one record).  qlora_profile_stop synchronises those events, disables the
+ * recording and writes up to max_entries aggregated rows: names (48 bytes
+ * each, NUL-terminated), total milliseconds, number of records and number of
+ * kernel launches; it returns the number of rows written.
+ */
+QLORA_API void qlora_profile_start(void);
+QLORA_API int qlora_profile_stop(int max_entries, char* names, float* total_ms, int* calls, int* launches);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLORA_H */

@@ -81,10 +81,16 @@ def bf16_bits(x: np.ndarray) -> np.ndarray:
     return (x.view(np.uint32) >> 16).astype(np.uint16)
 
 
-def _nearest_index(values: np.ndarray, levels: np.ndarray) -> np.ndarray:
-    """argmin_i |values - levels[i]| in float64, first (lowest) index on ties."""
-    d = np.abs(values.astype(np.float64)[:, None] - levels.astype(np.float64)[None, :])
-    return np.argmin(d, axis=1)
+def _nearest_index(values: np.ndarray, levels: np.ndarray, chunk: int = 1 << 20) -> np.ndarray:
+    """argmin_i |values - levels[i]| in float64, first (lowest) index on ties.
+
+    Evaluated in slices of ``chunk`` values only to bound memory."""
+    lv = levels.astype(np.float64)[None, :]
+    out = np.empty(values.size, dtype=np.int64)
+    for s in range(0, values.size, chunk):
+        d = np.abs(values[s:s + chunk].astype(np.float64)[:, None] - lv)
+        out[s:s + chunk] = np.argmin(d, axis=1)
+    return out
 
 
 def _level2_table() -> np.ndarray:

@@ -1,0 +1,111 @@
+"""Host-side checks of the C-ABI library that need no GPU: it loads, exports
+every function include/qlora.h declares, and rejects invalid calls on the
+host before anything is launched (fake pointers are never dereferenced)."""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import bit_quantized_lora_quantize_b200 as q
+from bit_quantized_lora_quantize_b200 import build as qbuild
+from oracle import nf4_codebook
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    qbuild.build()
+    return q.lib()
+
+
+def declared_functions():
+    with open(os.path.join(ROOT, "include", "qlora.h")) as f:
+        src = f.read()
+    return re.findall(r"QLORA_API\s+[\w\s\*]+?\b(qlora_\w+)\s*\(", src)
+
+
+def test_header_declares_the_boundary():
+    names = set(declared_functions())
+    for must in ("qlora_quantize_nf4", "qlora_dequantize_nf4", "qlora_linear_fwd", "qlora_linear_bwd",
+                 "qlora_workspace_bytes", "qlora_check_status", "qlora_nf4_codebook", "qlora_status_string"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+        assert ctypes.cast(getattr(L, name), ctypes.c_void_p).value
+
+
+def test_codebook_matches_oracle_in_float32(L):
+    np.testing.assert_array_equal(np.array(q.qlora_nf4_codebook(), dtype=np.float32), nf4_codebook())
+
+
+def test_status_strings(L):
+    for s in range(7):
+        assert L.qlora_status_string(s)
+
+
+FAKE = 1 << 20  # aligned, never dereferenced: every call below fails validation first
+
+
+def fwd(L, **kw):
+    a = dict(X=FAKE, M=16, K=256, N=256, codes=FAKE, aq=FAKE, sc=FAKE, A=FAKE, B=FAKE, r=8, s=2.0, Y=FAKE,
+             T=FAKE, ws=FAKE, nws=1 << 30, st=None)
+    a.update(kw)
+    return L.qlora_linear_fwd(a["X"], a["M"], a["K"], a["N"], a["codes"], a["aq"], a["sc"], a["A"], a["B"], a["r"],
+                              a["s"], a["Y"], a["T"], a["ws"], a["nws"], a["st"])
+
+
+def test_linear_fwd_validation(L):
+    assert fwd(L, X=None) == 1
+    assert fwd(L, s=float("nan")) == 1
+    assert fwd(L, M=0) == 1
+    assert fwd(L, K=100) == 3          # K % 64 != 0
+    assert fwd(L, N=260) == 3          # N % 8 != 0
+    assert fwd(L, r=12) == 3           # r % 8 != 0
+    assert fwd(L, r=136) == 3          # r > 128
+    assert fwd(L, X=FAKE + 8) == 2     # misaligned
+    assert fwd(L, ws=None) == 4
+    assert fwd(L, nws=16) == 4
+
+
+def test_linear_bwd_validation(L):
+    P = FAKE
+    base = [P, P, P, 16, 256, 256, P, P, P, P, P, 8, 2.0, P, P, P, P, 1 << 30, None]
+    assert L.qlora_linear_bwd(*base[:13], None, *base[14:]) == 1
+    bad = list(base)
+    bad[4] = 96
+    assert L.qlora_linear_bwd(*bad) == 3
+    bad = list(base)
+    bad[14] = P + 4
+    assert L.qlora_linear_bwd(*bad) == 2
+    bad = list(base)
+    bad[17] = 64
+    assert L.qlora_linear_bwd(*bad) == 4
+
+
+def test_codec_validation(L):
+    assert L.qlora_quantize_nf4(None, 64, FAKE, FAKE, FAKE, None) == 1
+    assert L.qlora_quantize_nf4(FAKE, 0, FAKE, FAKE, FAKE, None) == 1
+    assert L.qlora_quantize_nf4(FAKE + 2, 64, FAKE, FAKE, FAKE, None) == 2
+    assert L.qlora_dequantize_nf4(FAKE, FAKE, FAKE, -5, FAKE, None) == 1
+    assert L.qlora_dequantize_nf4(FAKE, FAKE, FAKE + 2, 64, FAKE, None) == 2
+
+
+def test_workspace_bytes(L):
+    assert q.qlora_workspace_bytes(16, 256, 256, 8) > 256
+    assert q.qlora_workspace_bytes(16, 100, 256, 8) == 0
+    a = q.qlora_workspace_bytes(4096, 4096, 4096, 64)
+    b = q.qlora_workspace_bytes(8192, 4096, 4096, 64)
+    assert b >= a > 4096 * 64 * 2
+
+
+def test_product_path_has_no_cpu_fallback():
+    import torch
+    with pytest.raises(ValueError):
+        q.qlora_quantize_nf4(torch.zeros(64, dtype=torch.bfloat16))
