@@ -177,7 +177,7 @@ def run_ours(args, rank, world, local_rank):
     import torch.distributed as dist
 
     import bit_quantized_lora_quantize_b200 as q
-    from bit_quantized_lora_quantize_b200 import build as qbuild, synthetic
+    from bit_quantized_lora_quantize_b200 import build as qbuild, dp, synthetic
 
     qbuild.build()
     dev = torch.device("cuda", local_rank)
@@ -194,16 +194,14 @@ def run_ours(args, rank, world, local_rank):
     dA = torch.empty(K, r, dtype=torch.float32, device=dev)
     dB = torch.empty(r, N, dtype=torch.float32, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # > L2 (126 MB)
-    grads = torch.empty(K * r + r * N, dtype=torch.float32, device=dev)
+    reducer = dp.AdapterGradReducer(K, N, r, dev) if world > 1 else None
 
     def step():
         Wp = q.qlora_quantize_nf4(W)
         q.qlora_linear_fwd(X, Wp, A, B, s, workspace=ws, Y=Y, T_save=T)
         q.qlora_linear_bwd(dY, X, T, Wp, A, B, s, workspace=ws, dX=dX, dA=dA, dB=dB)
-        if world > 1:
-            grads[:K * r].copy_(dA.view(-1))
-            grads[K * r:].copy_(dB.view(-1))
-            dist.all_reduce(grads)
+        if reducer is not None:
+            reducer(dA, dB)
         return Wp
 
     for _ in range(max(3, args.warmup)):
