@@ -1,0 +1,103 @@
+// Forward of the LoRA linear layer for callers that cannot allocate device
+// memory.
+//
+// Some callers cannot call cudaMalloc or any allocating routine: code that
+// runs where the allocator must not be touched (inside a memory-pool or
+// allocator callback, under a framework that forbids allocation on its hot
+// path, or in an embedding that owns all device memory up front).  They can
+// still pass their own inputs and outputs, but not the workspace that
+// qlora_linear_fwd needs.  qlora_linear_fwd_noalloc gives them the same
+// forward with its scratch taken from one fixed array in this file instead.
+//
+// The array is a file-scope __device__ variable of kNoAllocScratchBytes; every
+// GPU that loads this library keeps it for the life of the process.  Host
+// code cannot use the array's name as a device address, so the first call on
+// each device (with that device current) asks the runtime for the address
+// with cudaGetSymbolAddress and keeps it; that first call should therefore
+// come before any stream capture on that device.  All calls on a device share
+// the array and it keeps the previous call's contents: each call clears the
+// status word it needs at zero and overwrites everything else it reads, and
+// calls that overlap on the GPU (different streams, or different host threads
+// without ordering) race on it.
+#include <cstdint>
+#include <mutex>
+
+#include <cuda_runtime.h>
+
+#include "../../include/qlora.h"
+#include "kernels.h"
+#include "nf4_host.h"
+
+namespace qlora {
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB per device
+constexpr int kMaxDevices = 64;
+constexpr size_t kStatusBytes = 256;
+
+__device__ __align__(256) unsigned char g_fwd_scratch[kNoAllocScratchBytes];
+
+std::mutex g_setup_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+size_t round_up256(size_t v) { return (v + 255) / 256 * 256; }
+
+// Device address of the scratch array on the current device (set up once).
+cudaError_t scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> g(g_setup_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_fwd_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+
+}  // namespace qlora
+
+using namespace qlora;
+
+extern "C" qlora_status qlora_linear_fwd_noalloc(const uint16_t* X, int64_t M, int64_t K, int64_t N,
+                                                 const uint8_t* codes, const uint8_t* absmax_q,
+                                                 const float* absmax_scale, const uint16_t* A, const uint16_t* B,
+                                                 int32_t r, float scale, uint16_t* Y, float* T_save, void* stream) {
+  if (!X || !codes || !absmax_q || !absmax_scale || !A || !B || !Y || !T_save) return QLORA_ERR_INVALID_ARG;
+  if (!(scale == scale) || scale - scale != 0.0f) return QLORA_ERR_INVALID_ARG;  // NaN or infinite
+  if (M <= 0 || K <= 0 || N <= 0 || r <= 0) return QLORA_ERR_INVALID_ARG;
+  if (M >= (int64_t(1) << 31) || K >= (int64_t(1) << 31) || N >= (int64_t(1) << 31)) return QLORA_ERR_UNSUPPORTED;
+  if (K % 64 != 0 || N % 8 != 0 || r % 8 != 0 || r > 128) return QLORA_ERR_UNSUPPORTED;
+  const uintptr_t mis = reinterpret_cast<uintptr_t>(X) | reinterpret_cast<uintptr_t>(codes) |
+                        reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(B) |
+                        reinterpret_cast<uintptr_t>(Y) | reinterpret_cast<uintptr_t>(T_save);
+  if ((mis & 15u) || (reinterpret_cast<uintptr_t>(absmax_scale) & 3u)) return QLORA_ERR_ALIGNMENT;
+
+  // Scratch layout: [status word][T pair: bf16 M x 2rp][split partials of T].
+  const size_t pair_bytes = round_up256(static_cast<size_t>(M) * 2 * lora_pad(r) * 2);
+  const size_t part_bytes = round_up256(plan_skinny(SkinnyKind::kXA, M, K, N, r).partial_bytes);
+  if (kStatusBytes + pair_bytes + part_bytes > kNoAllocScratchBytes) return QLORA_ERR_WORKSPACE;
+
+  void* base = nullptr;
+  cudaError_t e = scratch_address(&base);
+  if (e != cudaSuccess) return QLORA_ERR_CUDA;
+  unsigned char* ws = static_cast<unsigned char*>(base);
+  int* status = reinterpret_cast<int*>(ws);
+  uint16_t* Tpair = reinterpret_cast<uint16_t*>(ws + kStatusBytes);
+  float* partial = reinterpret_cast<float*>(ws + kStatusBytes + pair_bytes);
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  e = cudaMemsetAsync(status, 0, sizeof(int), st);
+  if (e == cudaSuccess)
+    e = launch_skinny(SkinnyKind::kXA, X, A, M, K, N, r, scale, SkinnyOut{T_save, Tpair}, partial, status, st);
+  if (e == cudaSuccess)
+    e = launch_fused_fwd(X, codes, absmax_q, absmax_scale, Tpair, B, M, K, N, r, Y, status, nf4_params(), st);
+  return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}

@@ -31,6 +31,8 @@ _SIGS = {
                                         _P, _P, _P, ctypes.c_size_t, _P]),
     "qlora_linear_bwd": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P, _P, ctypes.c_int32,
                                         ctypes.c_float, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "qlora_linear_fwd_noalloc": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, ctypes.c_int32,
+                                                ctypes.c_float, _P, _P, _P]),
     "qlora_workspace_bytes": (ctypes.c_size_t, [_I64, _I64, _I64, ctypes.c_int32]),
     "qlora_check_status": (ctypes.c_int, [_P, _P]),
     "qlora_nf4_codebook": (None, [ctypes.POINTER(ctypes.c_float)]),
@@ -176,6 +178,20 @@ def qlora_linear_fwd(X: torch.Tensor, W: PackedNF4, A: torch.Tensor, B: torch.Te
     return Y, T_save
 
 
+def qlora_linear_fwd_noalloc(X: torch.Tensor, W: PackedNF4, A: torch.Tensor, B: torch.Tensor, scale: float,
+                             Y: torch.Tensor, T_save: torch.Tensor):
+    """Forward into caller-provided Y and T_save with no workspace: the
+    library takes its scratch from a fixed device array (see include/qlora.h)."""
+    M, K = X.shape
+    N = W.shape[0]
+    r = A.shape[1]
+    _require_cuda(X, A, B, W.codes, Y, T_save)
+    _check("qlora_linear_fwd_noalloc", lib().qlora_linear_fwd_noalloc(
+        _ptr(X), M, K, N, _ptr(W.codes), _ptr(W.absmax_q), _ptr(W.absmax_scale), _ptr(A), _ptr(B), r,
+        float(scale), _ptr(Y), _ptr(T_save), _stream()))
+    return Y, T_save
+
+
 def qlora_linear_bwd(dY: torch.Tensor, X: torch.Tensor, T_save: torch.Tensor, W: PackedNF4, A: torch.Tensor,
                      B: torch.Tensor, scale: float, workspace: torch.Tensor | None = None,
                      dX: torch.Tensor | None = None, dA: torch.Tensor | None = None, dB: torch.Tensor | None = None):
@@ -224,4 +240,5 @@ def qlora_profile_stop(max_entries: int = 32) -> dict:
 
 __all__ = ["qlora_profile_start", "qlora_profile_stop", "LIB_PATH", "lib", "QloraError", "PackedNF4", "packed_sizes", "qlora_nf4_codebook", "qlora_quantize_nf4",
            "qlora_dequantize_nf4", "qlora_workspace_bytes", "new_workspace", "qlora_linear_fwd", "qlora_linear_bwd",
+           "qlora_linear_fwd_noalloc",
            "qlora_check_status"]

@@ -148,6 +148,33 @@ QLORA_API qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, c
                               const uint16_t* A, const uint16_t* B, int32_t r, float scale, uint16_t* dX, float* dA,
                               float* dB, void* workspace, size_t ws_bytes, void* stream);
 
+/*
+ * qlora_linear_fwd without a workspace argument, for callers that cannot
+ * allocate device memory (code running inside an allocator or memory-pool
+ * callback, on a path where the framework forbids allocation, or in an
+ * embedding that owns all device memory up front).  The QLoRA pages have no
+ * counterpart to this call; it exists for those callers only.
+ *   Same arguments, outputs, supported shapes and results as
+ *   qlora_linear_fwd, minus workspace/ws_bytes.  The call allocates nothing:
+ *   its scratch is one fixed 16 MiB device array inside this library, which
+ *   every GPU that loads the library keeps until the process exits.
+ *   - Shapes whose forward scratch (status word + bf16 pair of T + split
+ *     partials of T) exceeds 16 MiB return QLORA_ERR_WORKSPACE and launch
+ *     nothing; the 4096 x 4096, 4096-token, r = 64 layer needs about 11.5 MiB.
+ *   - The first call on a device (with that device current, and `stream`
+ *     belonging to it) looks up the array's device address once; make that
+ *     first call before any stream capture on that device.
+ *   - All calls on a device share the array.  Calls that may overlap on the
+ *     GPU (other streams, or host threads without ordering) race and must be
+ *     serialised by the caller.
+ *   - Each call clears the status word it uses; a pipeline timeout inside
+ *     this call is not reported (qlora_check_status needs a workspace).
+ */
+QLORA_API qlora_status qlora_linear_fwd_noalloc(const uint16_t* X, int64_t M, int64_t K, int64_t N,
+                                                const uint8_t* codes, const uint8_t* absmax_q,
+                                                const float* absmax_scale, const uint16_t* A, const uint16_t* B,
+                                                int32_t r, float scale, uint16_t* Y, float* T_save, void* stream);
+
 /* Workspace bytes needed by qlora_linear_fwd / qlora_linear_bwd for these sizes
  * (0 for an unsupported shape). */
 QLORA_API size_t qlora_workspace_bytes(int64_t M, int64_t K, int64_t N, int32_t r);
