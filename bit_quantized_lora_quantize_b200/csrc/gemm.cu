@@ -38,9 +38,8 @@ namespace qlora {
 enum BKind : int { kBTmaK = 0, kBTmaMN = 1, kBNf4K = 2, kBNf4MN = 3 };
 enum EpiKind : int { kEpiBf16 = 0, kEpiPartial = 1 };
 
-constexpr int kBM = 128;
+constexpr int kBM = 128;                // rows of one tcgen05.mma (cta_group::1)
 constexpr int kBK = 64;
-constexpr int kABytes = kBM * kBK * 2;  // 16 KB
 constexpr int kCodeBytes = 8192;        // 256 x 32 B (Y) or 64 x 128 B (dX)
 
 struct GemmArgs {
@@ -61,9 +60,10 @@ struct GemmArgs {
   Nf4Params nf4;
 };
 
-template <int BN, int STAGES, int BK_KIND>
+template <int BM, int BN, int STAGES, int BK_KIND>
 struct SmemLayout {
   static constexpr bool kDecode = (BK_KIND == kBNf4K || BK_KIND == kBNf4MN);
+  static constexpr int kABytes = BM * kBK * 2;
   static constexpr int kBBytes = BN * kBK * 2;
   static constexpr int kCBytes = kDecode ? kCodeBytes : 0;
   static constexpr int kA = 0;
@@ -87,16 +87,21 @@ __device__ __forceinline__ void sts128(uint8_t* p, uint32_t a, uint32_t b, uint3
   *reinterpret_cast<uint4*>(p) = make_uint4(a, b, c, d);
 }
 
-template <int BN, int STAGES, bool A_MN, int BK_KIND, bool B2_MN, int EPI>
+template <int BM, int BN, int STAGES, bool A_MN, int BK_KIND, bool B2_MN, int EPI>
 __global__ void __launch_bounds__((BK_KIND == kBNf4K || BK_KIND == kBNf4MN) ? 384 : 256, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
                 const GemmArgs args) {
-  using L = SmemLayout<BN, STAGES, BK_KIND>;
+  using L = SmemLayout<BM, BN, STAGES, BK_KIND>;
   constexpr bool kDecode = L::kDecode;
   constexpr bool kBMN = (BK_KIND == kBTmaMN || BK_KIND == kBNf4MN);
-  constexpr uint32_t kTmemCols = TmemCols<BN>::value;
+  constexpr int kHalves = BM / kBM;  // MMAs per K step sharing one B tile
+  constexpr uint32_t kAccCols = TmemCols<BN>::value;
+  constexpr uint32_t kTmemCols = kAccCols * kHalves;
+  constexpr int kABytes = L::kABytes;
   constexpr int kDecoderWarps = 8;
+  static_assert(BM == 128 || (BM == 256 && BN == 256 && !A_MN), "256-row tiles: fused kernels only");
+  static_assert(kTmemCols <= 512, "TMEM budget");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -162,7 +167,7 @@ __global__ void __launch_bounds__((BK_KIND == kBNf4K || BK_KIND == kBNf4MN) ? 38
           const int kb = kb_begin + i;
           mbar_arrive_expect_tx(&full[s], kABytes + (kDecode ? kCodeBytes : L::kBBytes));
           if (!A_MN) {
-            tma_load_2d(&tmA, &full[s], a_dst, kb * kBK, tile_m * kBM);
+            tma_load_2d(&tmA, &full[s], a_dst, kb * kBK, tile_m * BM);
           } else {
             tma_load_2d(&tmA, &full[s], a_dst, tile_m * kBM, kb * kBK);
             tma_load_2d(&tmA, &full[s], a_dst + 8192, tile_m * kBM + 64, kb * kBK);
@@ -185,7 +190,7 @@ __global__ void __launch_bounds__((BK_KIND == kBNf4K || BK_KIND == kBNf4MN) ? 38
           const int lk = i - num_kb;
           const int lb = (lk * kBK) % args.lora_mod;
           mbar_arrive_expect_tx(&full[s], kABytes + 256 * kBK * 2);
-          tma_load_2d(&tmA2, &full[s], a_dst, lk * kBK, tile_m * kBM);
+          tma_load_2d(&tmA2, &full[s], a_dst, lk * kBK, tile_m * BM);
           if (B2_MN) {
 #pragma unroll
             for (int a = 0; a < 4; ++a) tma_load_2d(&tmB2, &full[s], b_dst + a * 8192, tile_n * 256 + a * 64, lb);
@@ -233,7 +238,13 @@ __global__ void __launch_bounds__((BK_KIND == kBNf4K || BK_KIND == kBNf4MN) ? 38
             bdesc = B2_MN ? smem_desc_sw128(b_base + kk * 2048, 8192, 1024) : smem_desc_sw128(b_base + kk * 32, 16, 1024);
             idesc = idesc_lora;
           }
-          umma_bf16(tmem_acc, adesc, bdesc, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+          const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+          umma_bf16(tmem_acc, adesc, bdesc, idesc, acc);
+          if (kHalves == 2) {
+            // Rows 128..255 of the A tile start 16 atoms (16 KB) further on.
+            const uint64_t adesc2 = smem_desc_sw128(a_base + 16384 + kk * 32, 16, 1024);
+            umma_bf16(tmem_acc + kAccCols, adesc2, bdesc, idesc, acc);
+          }
         }
         umma_commit(&empty[s]);
       }
@@ -350,14 +361,15 @@ __global__ void __launch_bounds__((BK_KIND == kBNf4K || BK_KIND == kBNf4MN) ? 38
       }
     }
     // ------------------------------------------------------------ epilogue
-    if (warp < 8) {
+    if (warp < 4 + 4 * kHalves) {
       const WaitCtx ctx{abort_flag, args.status, 4};
-      const int q = warp & 3;
+      const int q = warp & 3;           // TMEM lane group this warp may access
+      const int h = (warp - 4) >> 2;    // accumulator half (256-row tiles)
       const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(acc_full, 0, ctx));
       tc_fence_after();
       if (ok) {
-        const int row = tile_m * kBM + q * 32 + lane;
-        const uint32_t t_row = tmem_acc + (static_cast<uint32_t>(q * 32) << 16);
+        const int row = tile_m * BM + h * kBM + q * 32 + lane;
+        const uint32_t t_row = tmem_acc + (static_cast<uint32_t>(q * 32) << 16) + h * kAccCols;
 #pragma unroll 1
         for (int cc = 0; cc < BN / 32; ++cc) {
           uint32_t v[32];
@@ -380,7 +392,7 @@ __global__ void __launch_bounds__((BK_KIND == kBNf4K || BK_KIND == kBNf4MN) ? 38
               }
             }
           } else {
-            const int64_t rows_pad = static_cast<int64_t>(gridDim.y) * kBM;
+            const int64_t rows_pad = static_cast<int64_t>(gridDim.y) * BM;
             float* dst = args.partial + (static_cast<int64_t>(split) * rows_pad + row) * BN + cc * 32;
 #pragma unroll
             for (int g = 0; g < 8; ++g)
@@ -469,11 +481,11 @@ __global__ void split_pair_kernel(const float* __restrict__ v, int64_t rows, int
 }
 
 // ----------------------------------------------------------------- host side
-template <int BN, int STAGES, bool A_MN, int BK_KIND, bool B2_MN, int EPI>
+template <int BM, int BN, int STAGES, bool A_MN, int BK_KIND, bool B2_MN, int EPI>
 static cudaError_t launch_gemm(dim3 grid, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2,
                                const CUtensorMap& b2, const GemmArgs& args, cudaStream_t stream) {
-  using L = SmemLayout<BN, STAGES, BK_KIND>;
-  auto kern = gemm_kernel<BN, STAGES, A_MN, BK_KIND, B2_MN, EPI>;
+  using L = SmemLayout<BM, BN, STAGES, BK_KIND>;
+  auto kern = gemm_kernel<BM, BN, STAGES, A_MN, BK_KIND, B2_MN, EPI>;
   static_assert(L::kDynamic <= 232448, "shared memory budget");
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kDynamic);
   if (e != cudaSuccess) return e;
@@ -482,16 +494,17 @@ static cudaError_t launch_gemm(dim3 grid, const CUtensorMap& a, const CUtensorMa
   return cudaGetLastError();
 }
 
-constexpr int kFusedStages = 4;
+constexpr int kFusedBM = 256;
+constexpr int kFusedStages = 3;
 
 cudaError_t launch_fused_fwd(const uint16_t* X, const uint8_t* codes, const uint8_t* absmax_q,
                              const float* absmax_scale, const uint16_t* Tpair, const uint16_t* B, int64_t M, int64_t K,
                              int64_t N, int r, uint16_t* Y, int* status, const Nf4Params& P, cudaStream_t stream) {
   const int rp = lora_pad(r);
   CUtensorMap mX, mC, mT, mB;
-  if (!make_map_2d(&mX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, K * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+  if (!make_map_2d(&mX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, K * 2, 64, kFusedBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map_2d(&mC, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, K / 2, N, K / 2, 32, 256, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !make_map_2d(&mT, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Tpair, 2 * rp, M, static_cast<int64_t>(rp) * 4, 64, 128,
+      !make_map_2d(&mT, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Tpair, 2 * rp, M, static_cast<int64_t>(rp) * 4, 64, kFusedBM,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map_2d(&mB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, B, N, r, N * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
@@ -510,8 +523,8 @@ cudaError_t launch_fused_fwd(const uint16_t* X, const uint8_t* codes, const uint
   args.w_cols = K;
   args.status = status;
   args.nf4 = P;
-  dim3 grid(static_cast<unsigned>((N + 255) / 256), static_cast<unsigned>((M + kBM - 1) / kBM), 1);
-  return launch_gemm<256, kFusedStages, false, kBNf4K, true, kEpiBf16>(grid, mX, mC, mT, mB, args, stream);
+  dim3 grid(static_cast<unsigned>((N + 255) / 256), static_cast<unsigned>((M + kFusedBM - 1) / kFusedBM), 1);
+  return launch_gemm<kFusedBM, 256, kFusedStages, false, kBNf4K, true, kEpiBf16>(grid, mX, mC, mT, mB, args, stream);
 }
 
 cudaError_t launch_fused_dx(const uint16_t* dY, const uint8_t* codes, const uint8_t* absmax_q,
@@ -519,9 +532,9 @@ cudaError_t launch_fused_dx(const uint16_t* dY, const uint8_t* codes, const uint
                             int64_t N, int r, uint16_t* dX, int* status, const Nf4Params& P, cudaStream_t stream) {
   const int rp = lora_pad(r);
   CUtensorMap mD, mC, mU, mA;
-  if (!make_map_2d(&mD, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dY, N, M, N * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+  if (!make_map_2d(&mD, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dY, N, M, N * 2, 64, kFusedBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map_2d(&mC, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, K / 2, N, K / 2, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_2d(&mU, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Upair, 2 * rp, M, static_cast<int64_t>(rp) * 4, 64, 128,
+      !make_map_2d(&mU, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Upair, 2 * rp, M, static_cast<int64_t>(rp) * 4, 64, kFusedBM,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map_2d(&mA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, r, K, static_cast<int64_t>(r) * 2, 64, 256,
                    CU_TENSOR_MAP_SWIZZLE_128B))
@@ -541,8 +554,9 @@ cudaError_t launch_fused_dx(const uint16_t* dY, const uint8_t* codes, const uint
   args.w_cols = K;
   args.status = status;
   args.nf4 = P;
-  dim3 grid(static_cast<unsigned>((K + 255) / 256), static_cast<unsigned>((M + kBM - 1) / kBM), 1);
-  return launch_gemm<256, kFusedStages, false, kBNf4MN, false, kEpiBf16>(grid, mD, mC, mU, mA, args, stream);
+  dim3 grid(static_cast<unsigned>((K + 255) / 256), static_cast<unsigned>((M + kFusedBM - 1) / kFusedBM), 1);
+  return launch_gemm<kFusedBM, 256, kFusedStages, false, kBNf4MN, false, kEpiBf16>(grid, mD, mC, mU, mA, args,
+                                                                                    stream);
 }
 
 // ------------------------------------------------------------ skinny products
@@ -586,7 +600,8 @@ static cudaError_t launch_skinny_bn(const SkinnyPlan& p, const CUtensorMap& a, c
   args.lora_mod = 64;
   args.partial = partial;
   args.status = status;
-  return launch_gemm<BN, 4, A_MN, BK_KIND, false, kEpiPartial>(dim3(1, p.tiles, p.splits), a, b, a, b, args, stream);
+  return launch_gemm<kBM, BN, 4, A_MN, BK_KIND, false, kEpiPartial>(dim3(1, p.tiles, p.splits), a, b, a, b, args,
+                                                                    stream);
 }
 
 template <bool A_MN, int BK_KIND>
