@@ -413,53 +413,95 @@ __global__ void __launch_bounds__((BK_KIND == kBNf4K || BK_KIND == kBNf4MN) ? 38
 
 // Deterministic sum of the split partials (fixed order), then the output
 // conversion.  Producers (T, U) write the float32 value and its bf16 pair
-// (hi = bf16(v), lo = bf16(v - hi)); consumers (dA, dB) add the partial sums
-// of the hi and lo halves of their B operand.
+// (hi = bf16(v), lo = bf16(v - hi)); consumers (dA) add the partial sums of
+// the hi and lo halves of their B operand.  Each thread takes four adjacent
+// columns; the loads of four splits are issued before they are added.
+__device__ __forceinline__ float4 f4add(float4 a, float4 b) {
+  return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
+}
+
+__device__ __forceinline__ float4 sum_splits(const float* __restrict__ p, int splits, int64_t stride) {
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  int s = 0;
+  for (; s + 4 <= splits; s += 4) {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(p + s * stride));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(p + (s + 1) * stride));
+    const float4 c = __ldg(reinterpret_cast<const float4*>(p + (s + 2) * stride));
+    const float4 d = __ldg(reinterpret_cast<const float4*>(p + (s + 3) * stride));
+    acc = f4add(f4add(f4add(f4add(acc, a), b), c), d);
+  }
+  for (; s < splits; ++s) acc = f4add(acc, __ldg(reinterpret_cast<const float4*>(p + s * stride)));
+  return acc;
+}
+
+__device__ __forceinline__ void pair_bits(float v, uint16_t& hi, uint16_t& lo) {
+  const __nv_bfloat16 h = __float2bfloat16_rn(v);
+  const __nv_bfloat16 l = __float2bfloat16_rn(__fsub_rn(v, __bfloat162float(h)));
+  hi = *reinterpret_cast<const uint16_t*>(&h);
+  lo = *reinterpret_cast<const uint16_t*>(&l);
+}
+
 __global__ void skinny_reduce_kernel(const float* __restrict__ partial, int splits, int64_t rows_pad, int bn,
                                      int64_t rows, int r, int rp, float scale, int kind, float* __restrict__ f32,
                                      uint16_t* __restrict__ pair) {
   const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const bool producer = kind == static_cast<int>(SkinnyKind::kXA) || kind == static_cast<int>(SkinnyKind::kDyBt);
+  const int cols4 = (producer ? rp : r) / 4;
+  if (idx >= rows * cols4) return;
+  const int64_t row = idx / cols4;
+  const int j = static_cast<int>(idx % cols4) * 4;
+  const int64_t stride = rows_pad * bn;
+  const float* p = partial + row * bn + j;
   if (producer) {
-    if (idx >= rows * rp) return;
-    const int64_t row = idx / rp;
-    const int j = static_cast<int>(idx % rp);
-    uint16_t hi = 0, lo = 0;
+    uint16_t hi[4] = {0, 0, 0, 0}, lo[4] = {0, 0, 0, 0};
     if (j < r) {
-      float acc = 0.0f;
-      for (int s = 0; s < splits; ++s) acc += partial[(s * rows_pad + row) * bn + j];
-      const float v = __fmul_rn(scale, acc);
-      if (f32) f32[row * r + j] = v;
-      const __nv_bfloat16 h = __float2bfloat16_rn(v);
-      const __nv_bfloat16 l = __float2bfloat16_rn(__fsub_rn(v, __bfloat162float(h)));
-      hi = *reinterpret_cast<const uint16_t*>(&h);
-      lo = *reinterpret_cast<const uint16_t*>(&l);
+      const float4 a = sum_splits(p, splits, stride);
+      const float v[4] = {__fmul_rn(scale, a.x), __fmul_rn(scale, a.y), __fmul_rn(scale, a.z), __fmul_rn(scale, a.w)};
+      if (f32) *reinterpret_cast<float4*>(f32 + row * r + j) = make_float4(v[0], v[1], v[2], v[3]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) pair_bits(v[e], hi[e], lo[e]);
     }
-    pair[row * 2 * rp + j] = hi;
-    pair[row * 2 * rp + rp + j] = lo;
+    uint16_t* dst = pair + row * 2 * rp + j;
+    *reinterpret_cast<uint2*>(dst) = make_uint2(hi[0] | (uint32_t(hi[1]) << 16), hi[2] | (uint32_t(hi[3]) << 16));
+    *reinterpret_cast<uint2*>(dst + rp) =
+        make_uint2(lo[0] | (uint32_t(lo[1]) << 16), lo[2] | (uint32_t(lo[3]) << 16));
     return;
   }
-  if (idx >= rows * r) return;
-  int64_t row;
-  int j;
-  if (kind == static_cast<int>(SkinnyKind::kTtDy)) {
-    j = static_cast<int>(idx / rows);  // dB[j][n]: consecutive threads take consecutive n
-    row = idx % rows;
-  } else {
-    row = idx / r;
-    j = static_cast<int>(idx % r);
+  // kXtU: dA[row][j] = (sum of hi partials) + (sum of lo partials)
+  const float4 a = sum_splits(p, splits, stride);
+  const float4 b = sum_splits(p + rp, splits, stride);
+  *reinterpret_cast<float4*>(f32 + row * r + j) = f4add(a, b);
+}
+
+// dB[j][n] from partials laid out [split][n][2rp]: 32 rows (n) per block,
+// summed in split order, transposed through shared memory so both the loads
+// (along j) and the stores (along n) are coalesced.
+__global__ void skinny_reduce_t_kernel(const float* __restrict__ partial, int splits, int64_t rows_pad, int bn,
+                                       int64_t rows, int r, int rp, float* __restrict__ out) {
+  extern __shared__ float tile[];  // [32][r + 1]
+  const int64_t n0 = static_cast<int64_t>(blockIdx.x) * 32;
+  const int64_t stride = rows_pad * bn;
+  const int c4 = r / 4;
+  for (int t = threadIdx.x; t < 32 * c4; t += blockDim.x) {
+    const int nl = t / c4;
+    const int j = (t % c4) * 4;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (n0 + nl < rows) {
+      const float* p = partial + (n0 + nl) * bn + j;
+      v = f4add(sum_splits(p, splits, stride), sum_splits(p + rp, splits, stride));
+    }
+    float* d = tile + nl * (r + 1) + j;
+    d[0] = v.x;
+    d[1] = v.y;
+    d[2] = v.z;
+    d[3] = v.w;
   }
-  float acc_hi = 0.0f, acc_lo = 0.0f;
-  for (int s = 0; s < splits; ++s) {
-    const float* p = partial + (s * rows_pad + row) * bn;
-    acc_hi += p[j];
-    acc_lo += p[rp + j];
+  __syncthreads();
+  for (int t = threadIdx.x; t < 32 * r; t += blockDim.x) {
+    const int j = t / 32;
+    const int nl = t % 32;
+    if (n0 + nl < rows) out[static_cast<int64_t>(j) * rows + n0 + nl] = tile[nl * (r + 1) + j];
   }
-  const float v = acc_hi + acc_lo;
-  if (kind == static_cast<int>(SkinnyKind::kTtDy))
-    f32[static_cast<int64_t>(j) * rows + row] = v;
-  else
-    f32[row * r + j] = v;
 }
 
 // bf16 pair of a float32 [rows x r] matrix (see skinny_reduce_kernel).
@@ -574,7 +616,9 @@ SkinnyPlan plan_skinny(SkinnyKind kind, int64_t M, int64_t K, int64_t N, int r) 
   SkinnyPlan p{};
   p.tiles = static_cast<int>(ceil_div(rows, kBM));
   const int64_t nkb = ceil_div(red, kBK);
-  const int64_t want = ceil_div(2 * 148, p.tiles);
+  // One wave: two 96 KB CTAs per SM on the 148 SMs of a B200; each split keeps
+  // at least four 64-deep stages.
+  const int64_t want = std::max<int64_t>(1, (2 * 148) / p.tiles);
   int64_t splits = std::max<int64_t>(1, std::min<int64_t>(want, std::max<int64_t>(1, nkb / 4)));
   p.kb_per_split = static_cast<int>(ceil_div(nkb, splits));
   p.splits = static_cast<int>(ceil_div(nkb, p.kb_per_split));
@@ -600,8 +644,10 @@ static cudaError_t launch_skinny_bn(const SkinnyPlan& p, const CUtensorMap& a, c
   args.lora_mod = 64;
   args.partial = partial;
   args.status = status;
-  return launch_gemm<kBM, BN, 4, A_MN, BK_KIND, false, kEpiPartial>(dim3(1, p.tiles, p.splits), a, b, a, b, args,
-                                                                    stream);
+  // 96 KB of stages per CTA so that two CTAs share an SM.
+  constexpr int kStages = BN <= 64 ? 4 : 3;
+  return launch_gemm<kBM, BN, kStages, A_MN, BK_KIND, false, kEpiPartial>(dim3(1, p.tiles, p.splits), a, b, a, b,
+                                                                          args, stream);
 }
 
 template <bool A_MN, int BK_KIND>
@@ -663,11 +709,17 @@ cudaError_t launch_skinny(SkinnyKind kind, const uint16_t* P0, const uint16_t* P
   }
   if (e != cudaSuccess) return e;
   const bool producer = kind == SkinnyKind::kXA || kind == SkinnyKind::kDyBt;
-  const int64_t n_out = rows * (producer ? rp : r);
-  const int threads = 256;
-  skinny_reduce_kernel<<<static_cast<unsigned>(ceil_div(n_out, threads)), threads, 0, stream>>>(
-      partial, p.splits, static_cast<int64_t>(p.tiles) * kBM, p.bn, rows, r, rp, scale, static_cast<int>(kind),
-      out.f32, out.pair);
+  const int64_t rows_pad = static_cast<int64_t>(p.tiles) * kBM;
+  if (kind == SkinnyKind::kTtDy) {
+    const size_t smem = static_cast<size_t>(32) * (r + 1) * sizeof(float);
+    skinny_reduce_t_kernel<<<static_cast<unsigned>(ceil_div(rows, 32)), 256, smem, stream>>>(
+        partial, p.splits, rows_pad, p.bn, rows, r, rp, out.f32);
+  } else {
+    const int64_t n_out = rows * ((producer ? rp : r) / 4);
+    const int threads = 256;
+    skinny_reduce_kernel<<<static_cast<unsigned>(ceil_div(n_out, threads)), threads, 0, stream>>>(
+        partial, p.splits, rows_pad, p.bn, rows, r, rp, scale, static_cast<int>(kind), out.f32, out.pair);
+  }
   return cudaGetLastError();
 }
 

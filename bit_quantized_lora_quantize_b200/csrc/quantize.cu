@@ -11,12 +11,14 @@
 // reduction and no intermediate constant ever goes to HBM.  Loads are
 // coalesced 16-byte vectors staged in shared memory; each thread then owns
 // one 64-element block.
+#include <algorithm>
 #include <cstdint>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include "kernels.h"
 #include "nf4_device.cuh"
+#include "tensor_map.h"
 
 namespace qlora {
 
@@ -27,108 +29,158 @@ constexpr int kThreads = 256;
 
 // Shared tile: 256 blocks x 128 B.  Thread t reads its block's 16-byte chunk
 // j at position (j + t) mod 8 of the row, which spreads the eight lanes of a
-// quarter-warp over all banks.
+// quarter-warp over all banks (used by the dequantization kernel).
 __device__ __forceinline__ uint32_t chunk_pos(int row, int j) { return row * 128 + (((j + row) & 7) << 4); }
 
-__global__ void __launch_bounds__(kThreads) quantize_nf4_kernel(const uint16_t* __restrict__ W, int64_t numel,
-                                                                 uint8_t* __restrict__ codes,
-                                                                 uint8_t* __restrict__ absmax_q,
-                                                                 float* __restrict__ absmax_scale, Nf4Params P) {
-  __shared__ __align__(16) uint8_t tile[kGroupElems * 2];
-  __shared__ float warp_max[kThreads / 32];
+// Quantization, persistent: each CTA walks over groups with a two-deep TMA
+// pipeline.  The weight is viewed as [numel/64 rows x 64] bf16 (one absmax
+// block per row); a 256-row box lands with the 128-byte swizzle, so thread t
+// finds logical chunk j of its block at chunk position j ^ (t & 7) and the
+// eight lanes of a quarter-warp hit eight different bank groups.  The group
+// holding a partial last block (numel % 64 != 0) is staged with plain loads
+// in the same layout.
+constexpr int kQuantStages = 2;
+constexpr int kQuantSmem = kQuantStages * kGroupElems * 2 + 1024 + 256 * 4 + 128;
+
+__global__ void __launch_bounds__(kThreads, 3)
+    quantize_nf4_kernel(const __grid_constant__ CUtensorMap tmW, const uint16_t* __restrict__ W, int64_t numel,
+                        uint8_t* __restrict__ codes, uint8_t* __restrict__ absmax_q,
+                        float* __restrict__ absmax_scale, Nf4Params P) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* buf = smem;                                                   // 2 x 32 KB
+  float* lvl2 = reinterpret_cast<float*>(smem + kQuantStages * kGroupElems * 2);  // fp32(k/255)
+  uint64_t* bar = reinterpret_cast<uint64_t*>(lvl2 + 256);
+  float* warp_max = reinterpret_cast<float*>(bar + kQuantStages);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(warp_max + kThreads / 32);
   const int tid = threadIdx.x;
-  const int64_t base = static_cast<int64_t>(blockIdx.x) * kGroupElems;
-  const bool full = base + kGroupElems <= numel;
+  const WaitCtx ctx{abort_flag, nullptr, 5};
 
-  // Coalesced load of the group: chunk i (8 elements) -> block i / 8, chunk i % 8.
-#pragma unroll
-  for (int it = 0; it < 8; ++it) {
-    const int chunk = tid + it * kThreads;
-    const int64_t e0 = base + static_cast<int64_t>(chunk) * 8;
-    uint4 v;
-    if (full) {
-      v = __ldg(reinterpret_cast<const uint4*>(W + e0));
-    } else {
-      uint16_t h[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) h[e] = (e0 + e < numel) ? W[e0 + e] : static_cast<uint16_t>(0);
-      v.x = h[0] | (static_cast<uint32_t>(h[1]) << 16);
-      v.y = h[2] | (static_cast<uint32_t>(h[3]) << 16);
-      v.z = h[4] | (static_cast<uint32_t>(h[5]) << 16);
-      v.w = h[6] | (static_cast<uint32_t>(h[7]) << 16);
-    }
-    *reinterpret_cast<uint4*>(tile + chunk_pos(chunk >> 3, chunk & 7)) = v;
-  }
-  __syncthreads();
-
-  // This thread's block: 32 bf16 pairs.
-  uint32_t x[32];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const uint4 v = *reinterpret_cast<const uint4*>(tile + chunk_pos(tid, j));
-    x[4 * j + 0] = v.x;
-    x[4 * j + 1] = v.y;
-    x[4 * j + 2] = v.z;
-    x[4 * j + 3] = v.w;
-  }
-  // Block absmax (absent tail elements were loaded as zero).
-  __nv_bfloat162 mx = __floats2bfloat162_rn(0.0f, 0.0f);
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    uint32_t a = x[i] & 0x7FFF7FFFu;
-    mx = __hmax2(mx, *reinterpret_cast<__nv_bfloat162*>(&a));
-  }
-  const float c = fmaxf(__low2float(mx), __high2float(mx));
-
-  // Group maximum c1.
-  float m = c;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-  if ((tid & 31) == 0) warp_max[tid >> 5] = m;
-  __syncthreads();
-  float c1 = warp_max[0];
-#pragma unroll
-  for (int w = 1; w < kThreads / 32; ++w) c1 = fmaxf(c1, warp_max[w]);
-
-  const int64_t blk = static_cast<int64_t>(blockIdx.x) * kGroup + tid;
+  const int64_t groups = (numel + kGroupElems - 1) / kGroupElems;
   const int64_t nb = (numel + kBlock - 1) / kBlock;
-  if (blk < nb) {
-    // 8-bit code of c / c1: nearest fp32(k / 255), ties to the lower k.
-    uint32_t code2 = 0;
-    if (c1 > 0.0f) {
-      const float n2 = __fdiv_rn(c, c1);
-      int k0 = __float2int_rn(n2 * 255.0f);
-      k0 = max(2, min(253, k0));
-      double best = 4.0;
-#pragma unroll
-      for (int d = -2; d <= 2; ++d) {
-        const double dist = fabs(static_cast<double>(n2) - static_cast<double>(level2_value(k0 + d)));
-        if (dist < best) {
-          best = dist;
-          code2 = static_cast<uint32_t>(k0 + d);
+  const int64_t nbytes = (numel + 1) / 2;
+  const bool ragged_tail = (numel % kBlock) != 0;  // last group staged with plain loads
+
+  lvl2[tid] = level2_value(tid);
+  if (tid == 0) {
+    for (int s = 0; s < kQuantStages; ++s) mbar_init(&bar[s], 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  __syncthreads();
+
+  auto issue = [&](int64_t g, int stage) {
+    // Thread 0 only.  A group that needs plain loads is staged by all threads
+    // after the wait instead.
+    if (ragged_tail && g == groups - 1) {
+      mbar_arrive(&bar[stage]);
+      return;
+    }
+    mbar_arrive_expect_tx(&bar[stage], kGroupElems * 2);
+    tma_load_2d(&tmW, &bar[stage], buf + stage * kGroupElems * 2, 0, static_cast<int>(g * kGroup));
+  };
+
+  int it = 0;
+  int64_t g = blockIdx.x;
+  if (tid == 0 && g < groups) issue(g, 0);
+  for (; g < groups; g += gridDim.x, ++it) {
+    const int stage = it & 1;
+    const uint32_t phase = (it >> 1) & 1;
+    const int64_t gn = g + gridDim.x;
+    if (tid == 0 && gn < groups) issue(gn, stage ^ 1);
+    // Bounded wait: a copy that never lands ends the loop (the caller sees
+    // undefined codes) instead of hanging the device.
+    if (!__syncthreads_and(mbar_wait(&bar[stage], phase, ctx))) {
+      if (tid == 0 && gn < groups) {
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(&bar[stage ^ 1], ((it + 1) >> 1) & 1) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
         }
       }
+      break;
     }
-    absmax_q[blk] = static_cast<uint8_t>(code2);
-  }
-  if (tid == 0) absmax_scale[blockIdx.x] = c1;
-
-  // 4-bit codes of the block.
-  const Nf4Thresholds T = make_thresholds(P, c);
-  uint32_t out[8];
+    uint8_t* tile = buf + stage * kGroupElems * 2;
+    const int64_t base = g * kGroupElems;
+    if (ragged_tail && g == groups - 1) {
+      for (int chunk = tid; chunk < kGroupElems / 8; chunk += kThreads) {
+        const int64_t e0 = base + static_cast<int64_t>(chunk) * 8;
+        uint16_t h[8];
 #pragma unroll
-  for (int j = 0; j < 8; ++j)
-    out[j] = pack_codes8(encode_pair(T, x[4 * j]), encode_pair(T, x[4 * j + 1]), encode_pair(T, x[4 * j + 2]),
-                         encode_pair(T, x[4 * j + 3]));
+        for (int e = 0; e < 8; ++e) h[e] = (e0 + e < numel) ? W[e0 + e] : static_cast<uint16_t>(0);
+        const int row = chunk >> 3, c = chunk & 7;
+        *reinterpret_cast<uint4*>(tile + row * 128 + ((c ^ (row & 7)) << 4)) =
+            make_uint4(h[0] | (uint32_t(h[1]) << 16), h[2] | (uint32_t(h[3]) << 16), h[4] | (uint32_t(h[5]) << 16),
+                       h[6] | (uint32_t(h[7]) << 16));
+      }
+      __syncthreads();
+    }
 
-  const int64_t byte0 = (base + static_cast<int64_t>(tid) * kBlock) / 2;
-  const int64_t nbytes = (numel + 1) / 2;
-  if (byte0 + 32 <= nbytes) {
-    uint4* dst = reinterpret_cast<uint4*>(codes + byte0);
-    dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
-    dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
-  } else {
-    for (int b = 0; b < 32 && byte0 + b < nbytes; ++b) codes[byte0 + b] = static_cast<uint8_t>(out[b >> 2] >> (8 * (b & 3)));
+    // This thread's block: 32 bf16 pairs in element order.
+    uint32_t x[32];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint4 v = *reinterpret_cast<const uint4*>(tile + tid * 128 + ((j ^ (tid & 7)) << 4));
+      x[4 * j + 0] = v.x;
+      x[4 * j + 1] = v.y;
+      x[4 * j + 2] = v.z;
+      x[4 * j + 3] = v.w;
+    }
+    // Block absmax (elements beyond numel were staged as zero).
+    __nv_bfloat162 mx = __floats2bfloat162_rn(0.0f, 0.0f);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      uint32_t a = x[i] & 0x7FFF7FFFu;
+      mx = __hmax2(mx, *reinterpret_cast<__nv_bfloat162*>(&a));
+    }
+    const float c = fmaxf(__low2float(mx), __high2float(mx));
+
+    // Group maximum c1.
+    float m = c;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    if ((tid & 31) == 0) warp_max[tid >> 5] = m;
+    __syncthreads();  // also: every thread has read `tile`
+    float c1 = warp_max[0];
+#pragma unroll
+    for (int w = 1; w < kThreads / 32; ++w) c1 = fmaxf(c1, warp_max[w]);
+
+    const int64_t blk = g * kGroup + tid;
+    if (blk < nb) {
+      // 8-bit code of c / c1: nearest fp32(k / 255), ties to the lower k.
+      uint32_t code2 = 0;
+      if (c1 > 0.0f) {
+        const float n2 = __fdiv_rn(c, c1);
+        int k0 = __float2int_rn(n2 * 255.0f);
+        k0 = max(2, min(253, k0));
+        double best = 4.0;
+#pragma unroll
+        for (int d = -2; d <= 2; ++d) {
+          const double dist = fabs(static_cast<double>(n2) - static_cast<double>(lvl2[k0 + d]));
+          if (dist < best) {
+            best = dist;
+            code2 = static_cast<uint32_t>(k0 + d);
+          }
+        }
+      }
+      absmax_q[blk] = static_cast<uint8_t>(code2);
+    }
+    if (tid == 0) absmax_scale[g] = c1;
+
+    // 4-bit codes of the block.
+    const Nf4Thresholds T = make_thresholds(P, c);
+    uint32_t out[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      out[j] = pack_codes8(encode_pair(T, x[4 * j]), encode_pair(T, x[4 * j + 1]), encode_pair(T, x[4 * j + 2]),
+                           encode_pair(T, x[4 * j + 3]));
+    const int64_t byte0 = blk * (kBlock / 2);
+    if (byte0 + 32 <= nbytes) {
+      uint4* dst = reinterpret_cast<uint4*>(codes + byte0);
+      dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
+      dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
+    } else {
+      for (int b = 0; b < 32 && byte0 + b < nbytes; ++b)
+        codes[byte0 + b] = static_cast<uint8_t>(out[b >> 2] >> (8 * (b & 3)));
+    }
   }
 }
 
@@ -194,8 +246,25 @@ __global__ void __launch_bounds__(kThreads) dequantize_nf4_kernel(const uint8_t*
 cudaError_t launch_quantize_nf4(const uint16_t* W, int64_t numel, uint8_t* codes, uint8_t* absmax_q,
                                 float* absmax_scale, const Nf4Params& P, cudaStream_t stream) {
   const int64_t groups = (numel + kGroupElems - 1) / kGroupElems;
-  quantize_nf4_kernel<<<static_cast<unsigned>(groups), kThreads, 0, stream>>>(W, numel, codes, absmax_q,
-                                                                              absmax_scale, P);
+  const int64_t full_rows = numel / kBlock;
+  CUtensorMap map;
+  // A 2-D view needs at least one complete block; a smaller tensor is a
+  // single ragged group staged with plain loads (the map is then unused).
+  if (!make_map_2d(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, kBlock, full_rows > 0 ? full_rows : 1, kBlock * 2,
+                   kBlock, kGroup, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  static int sm_count = 0;
+  if (sm_count == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sm_count <= 0)
+      sm_count = 148;
+  }
+  cudaError_t e = cudaFuncSetAttribute(quantize_nf4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kQuantSmem);
+  if (e != cudaSuccess) return e;
+  const int64_t grid = std::min<int64_t>(groups, static_cast<int64_t>(sm_count) * 3);
+  quantize_nf4_kernel<<<static_cast<unsigned>(grid), kThreads, kQuantSmem, stream>>>(map, W, numel, codes, absmax_q,
+                                                                                      absmax_scale, P);
   return cudaGetLastError();
 }
 
