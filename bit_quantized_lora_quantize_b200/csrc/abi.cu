@@ -34,18 +34,18 @@ constexpr size_t kStatusBytes = 256;
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // Workspace: [status word (256 B)][T pair: bf16 M x 2rp][U pair: bf16 M x 2rp]
-//            [split partials (fp32)]
 struct WsLayout {
-  size_t t_off, u_off, part_off, total;
+  size_t t_off, u_off, total;
 };
 
 WsLayout ws_layout(int64_t M, int64_t K, int64_t N, int r) {
+  (void)K;
+  (void)N;
   WsLayout w{};
   const size_t pair_bytes = round_up(static_cast<size_t>(M) * 2 * lora_pad(r) * 2, 256);
   w.t_off = kStatusBytes;
   w.u_off = w.t_off + pair_bytes;
-  w.part_off = w.u_off + pair_bytes;
-  w.total = w.part_off + round_up(skinny_partial_bytes_max(M, K, N, r), 256);
+  w.total = w.u_off + pair_bytes;
   return w;
 }
 
@@ -188,14 +188,13 @@ qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, int64_t K, int64_t N
   if (!aligned16(workspace)) return QLORA_ERR_ALIGNMENT;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   int* status = reinterpret_cast<int*>(ws);
-  float* partial = reinterpret_cast<float*>(ws + wl.part_off);
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   const Nf4Params& P = nf4_params();
 
   uint16_t* Tpair = reinterpret_cast<uint16_t*>(ws + wl.t_off);
 
-  ProfScope p1(st, "lora_down_xa", 2);
-  cudaError_t e = launch_skinny(SkinnyKind::kXA, X, A, M, K, N, r, scale, SkinnyOut{T_save, Tpair}, partial, status, st);
+  ProfScope p1(st, "lora_down_xa", 1);
+  cudaError_t e = launch_skinny(SkinnyKind::kXA, X, A, M, K, N, r, scale, SkinnyOut{T_save, Tpair}, status, st);
   p1.done();
   if (e != cudaSuccess) return cuda_fail(e);
   ProfScope p2(st, "fused_nf4_fwd", 1);
@@ -225,27 +224,25 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float
   int* status = reinterpret_cast<int*>(ws);
   uint16_t* Tpair = reinterpret_cast<uint16_t*>(ws + wl.t_off);
   uint16_t* Upair = reinterpret_cast<uint16_t*>(ws + wl.u_off);
-  float* partial = reinterpret_cast<float*>(ws + wl.part_off);
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   const Nf4Params& P = nf4_params();
 
-  ProfScope p1(st, "lora_u_dybt", 2);
-  cudaError_t e = launch_skinny(SkinnyKind::kDyBt, dY, B, M, K, N, r, scale, SkinnyOut{nullptr, Upair}, partial,
-                                status, st);
+  ProfScope p1(st, "lora_u_dybt", 1);
+  cudaError_t e = launch_skinny(SkinnyKind::kDyBt, dY, B, M, K, N, r, scale, SkinnyOut{nullptr, Upair}, status, st);
   p1.done();
   if (e != cudaSuccess) return cuda_fail(e);
-  ProfScope p2(st, "lora_db_ttdy", 3);
+  ProfScope p2(st, "lora_db_ttdy", 2);
   e = launch_split_pair(T_save, M, r, Tpair, st);
   if (e == cudaSuccess)
-    e = launch_skinny(SkinnyKind::kTtDy, dY, Tpair, M, K, N, r, 1.0f, SkinnyOut{dB, nullptr}, partial, status, st);
+    e = launch_skinny(SkinnyKind::kTtDy, dY, Tpair, M, K, N, r, 1.0f, SkinnyOut{dB, nullptr}, status, st);
   p2.done();
   if (e != cudaSuccess) return cuda_fail(e);
   ProfScope p3(st, "fused_nf4_dx", 1);
   e = launch_fused_dx(dY, codes, absmax_q, absmax_scale, Upair, A, M, K, N, r, dX, status, P, st);
   p3.done();
   if (e != cudaSuccess) return cuda_fail(e);
-  ProfScope p4(st, "lora_da_xtu", 2);
-  e = launch_skinny(SkinnyKind::kXtU, X, Upair, M, K, N, r, 1.0f, SkinnyOut{dA, nullptr}, partial, status, st);
+  ProfScope p4(st, "lora_da_xtu", 1);
+  e = launch_skinny(SkinnyKind::kXtU, X, Upair, M, K, N, r, 1.0f, SkinnyOut{dA, nullptr}, status, st);
   p4.done();
   if (e != cudaSuccess) return cuda_fail(e);
   return QLORA_OK;
@@ -260,8 +257,7 @@ qlora_status qlora_check_status(void* workspace, void* stream) {
   e = cudaMemcpy(&word, workspace, sizeof(int), cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return cuda_fail(e);
   if (word == 0) return QLORA_OK;
-  const int zero = 0;
-  e = cudaMemcpy(workspace, &zero, sizeof(int), cudaMemcpyHostToDevice);
+  e = cudaMemset(workspace, 0, sizeof(int));
   if (e != cudaSuccess) return cuda_fail(e);
   return QLORA_ERR_TIMEOUT;
 }

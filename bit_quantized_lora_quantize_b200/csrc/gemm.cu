@@ -18,9 +18,6 @@
 // The LoRA term of the fused kernels is one (or, for r > 64, a few) extra
 // 64-deep reduction stage appended to the same TMEM accumulator:
 //   Y  = [X | T] [W'^T ; B]      dX = [dY | U] [W' ; A^T]
-// The rank-r "skinny" products use the same template with a TMA-fed B operand
-// and split the reduction across CTAs; a second kernel sums the splits in a
-// fixed order (deterministic, no float atomics).
 #include <algorithm>
 #include <cstdint>
 #include <cstdio>
@@ -411,117 +408,6 @@ __global__ void __launch_bounds__((BK_KIND == kBNf4K || BK_KIND == kBNf4MN) ? 38
   }
 }
 
-// Deterministic sum of the split partials (fixed order), then the output
-// conversion.  Producers (T, U) write the float32 value and its bf16 pair
-// (hi = bf16(v), lo = bf16(v - hi)); consumers (dA) add the partial sums of
-// the hi and lo halves of their B operand.  Each thread takes four adjacent
-// columns; the loads of four splits are issued before they are added.
-__device__ __forceinline__ float4 f4add(float4 a, float4 b) {
-  return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
-}
-
-__device__ __forceinline__ float4 sum_splits(const float* __restrict__ p, int splits, int64_t stride) {
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  int s = 0;
-  for (; s + 4 <= splits; s += 4) {
-    const float4 a = __ldg(reinterpret_cast<const float4*>(p + s * stride));
-    const float4 b = __ldg(reinterpret_cast<const float4*>(p + (s + 1) * stride));
-    const float4 c = __ldg(reinterpret_cast<const float4*>(p + (s + 2) * stride));
-    const float4 d = __ldg(reinterpret_cast<const float4*>(p + (s + 3) * stride));
-    acc = f4add(f4add(f4add(f4add(acc, a), b), c), d);
-  }
-  for (; s < splits; ++s) acc = f4add(acc, __ldg(reinterpret_cast<const float4*>(p + s * stride)));
-  return acc;
-}
-
-__device__ __forceinline__ void pair_bits(float v, uint16_t& hi, uint16_t& lo) {
-  const __nv_bfloat16 h = __float2bfloat16_rn(v);
-  const __nv_bfloat16 l = __float2bfloat16_rn(__fsub_rn(v, __bfloat162float(h)));
-  hi = *reinterpret_cast<const uint16_t*>(&h);
-  lo = *reinterpret_cast<const uint16_t*>(&l);
-}
-
-__global__ void skinny_reduce_kernel(const float* __restrict__ partial, int splits, int64_t rows_pad, int bn,
-                                     int64_t rows, int r, int rp, float scale, int kind, float* __restrict__ f32,
-                                     uint16_t* __restrict__ pair) {
-  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const bool producer = kind == static_cast<int>(SkinnyKind::kXA) || kind == static_cast<int>(SkinnyKind::kDyBt);
-  const int cols4 = (producer ? rp : r) / 4;
-  if (idx >= rows * cols4) return;
-  const int64_t row = idx / cols4;
-  const int j = static_cast<int>(idx % cols4) * 4;
-  const int64_t stride = rows_pad * bn;
-  const float* p = partial + row * bn + j;
-  if (producer) {
-    uint16_t hi[4] = {0, 0, 0, 0}, lo[4] = {0, 0, 0, 0};
-    if (j < r) {
-      const float4 a = sum_splits(p, splits, stride);
-      const float v[4] = {__fmul_rn(scale, a.x), __fmul_rn(scale, a.y), __fmul_rn(scale, a.z), __fmul_rn(scale, a.w)};
-      if (f32) *reinterpret_cast<float4*>(f32 + row * r + j) = make_float4(v[0], v[1], v[2], v[3]);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) pair_bits(v[e], hi[e], lo[e]);
-    }
-    uint16_t* dst = pair + row * 2 * rp + j;
-    *reinterpret_cast<uint2*>(dst) = make_uint2(hi[0] | (uint32_t(hi[1]) << 16), hi[2] | (uint32_t(hi[3]) << 16));
-    *reinterpret_cast<uint2*>(dst + rp) =
-        make_uint2(lo[0] | (uint32_t(lo[1]) << 16), lo[2] | (uint32_t(lo[3]) << 16));
-    return;
-  }
-  // kXtU: dA[row][j] = (sum of hi partials) + (sum of lo partials)
-  const float4 a = sum_splits(p, splits, stride);
-  const float4 b = sum_splits(p + rp, splits, stride);
-  *reinterpret_cast<float4*>(f32 + row * r + j) = f4add(a, b);
-}
-
-// dB[j][n] from partials laid out [split][n][2rp]: 32 rows (n) per block,
-// summed in split order, transposed through shared memory so both the loads
-// (along j) and the stores (along n) are coalesced.
-__global__ void skinny_reduce_t_kernel(const float* __restrict__ partial, int splits, int64_t rows_pad, int bn,
-                                       int64_t rows, int r, int rp, float* __restrict__ out) {
-  extern __shared__ float tile[];  // [32][r + 1]
-  const int64_t n0 = static_cast<int64_t>(blockIdx.x) * 32;
-  const int64_t stride = rows_pad * bn;
-  const int c4 = r / 4;
-  for (int t = threadIdx.x; t < 32 * c4; t += blockDim.x) {
-    const int nl = t / c4;
-    const int j = (t % c4) * 4;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (n0 + nl < rows) {
-      const float* p = partial + (n0 + nl) * bn + j;
-      v = f4add(sum_splits(p, splits, stride), sum_splits(p + rp, splits, stride));
-    }
-    float* d = tile + nl * (r + 1) + j;
-    d[0] = v.x;
-    d[1] = v.y;
-    d[2] = v.z;
-    d[3] = v.w;
-  }
-  __syncthreads();
-  for (int t = threadIdx.x; t < 32 * r; t += blockDim.x) {
-    const int j = t / 32;
-    const int nl = t % 32;
-    if (n0 + nl < rows) out[static_cast<int64_t>(j) * rows + n0 + nl] = tile[nl * (r + 1) + j];
-  }
-}
-
-// bf16 pair of a float32 [rows x r] matrix (see skinny_reduce_kernel).
-__global__ void split_pair_kernel(const float* __restrict__ v, int64_t rows, int r, int rp, uint16_t* __restrict__ pair) {
-  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (idx >= rows * rp) return;
-  const int64_t row = idx / rp;
-  const int j = static_cast<int>(idx % rp);
-  uint16_t hi = 0, lo = 0;
-  if (j < r) {
-    const float x = v[row * r + j];
-    const __nv_bfloat16 h = __float2bfloat16_rn(x);
-    const __nv_bfloat16 l = __float2bfloat16_rn(__fsub_rn(x, __bfloat162float(h)));
-    hi = *reinterpret_cast<const uint16_t*>(&h);
-    lo = *reinterpret_cast<const uint16_t*>(&l);
-  }
-  pair[row * 2 * rp + j] = hi;
-  pair[row * 2 * rp + rp + j] = lo;
-}
-
 // ----------------------------------------------------------------- host side
 template <int BM, int BN, int STAGES, bool A_MN, int BK_KIND, bool B2_MN, int EPI>
 static cudaError_t launch_gemm(dim3 grid, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2,
@@ -599,135 +485,6 @@ cudaError_t launch_fused_dx(const uint16_t* dY, const uint8_t* codes, const uint
   dim3 grid(static_cast<unsigned>((K + 255) / 256), static_cast<unsigned>((M + kFusedBM - 1) / kFusedBM), 1);
   return launch_gemm<kFusedBM, 256, kFusedStages, false, kBNf4MN, false, kEpiBf16>(grid, mD, mC, mU, mA, args,
                                                                                     stream);
-}
-
-// ------------------------------------------------------------ skinny products
-static int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
-
-SkinnyPlan plan_skinny(SkinnyKind kind, int64_t M, int64_t K, int64_t N, int r) {
-  int64_t rows, red;
-  switch (kind) {
-    case SkinnyKind::kXA: rows = M; red = K; break;
-    case SkinnyKind::kDyBt: rows = M; red = N; break;
-    case SkinnyKind::kTtDy: rows = N; red = M; break;
-    default: rows = K; red = M; break;
-  }
-  const bool producer = kind == SkinnyKind::kXA || kind == SkinnyKind::kDyBt;
-  SkinnyPlan p{};
-  p.tiles = static_cast<int>(ceil_div(rows, kBM));
-  const int64_t nkb = ceil_div(red, kBK);
-  // One wave: two 96 KB CTAs per SM on the 148 SMs of a B200; each split keeps
-  // at least four 64-deep stages.
-  const int64_t want = std::max<int64_t>(1, (2 * 148) / p.tiles);
-  int64_t splits = std::max<int64_t>(1, std::min<int64_t>(want, std::max<int64_t>(1, nkb / 4)));
-  p.kb_per_split = static_cast<int>(ceil_div(nkb, splits));
-  p.splits = static_cast<int>(ceil_div(nkb, p.kb_per_split));
-  p.bn = producer ? lora_pad(r) : 2 * lora_pad(r);
-  p.partial_bytes = static_cast<size_t>(p.splits) * p.tiles * kBM * p.bn * sizeof(float);
-  return p;
-}
-
-size_t skinny_partial_bytes_max(int64_t M, int64_t K, int64_t N, int r) {
-  size_t m = 0;
-  for (SkinnyKind k : {SkinnyKind::kXA, SkinnyKind::kDyBt, SkinnyKind::kTtDy, SkinnyKind::kXtU})
-    m = std::max(m, plan_skinny(k, M, K, N, r).partial_bytes);
-  return m;
-}
-
-template <int BN, bool A_MN, int BK_KIND>
-static cudaError_t launch_skinny_bn(const SkinnyPlan& p, const CUtensorMap& a, const CUtensorMap& b, int64_t red,
-                                    float* partial, int* status, cudaStream_t stream) {
-  GemmArgs args{};
-  args.nkb_total = static_cast<int>(ceil_div(red, kBK));
-  args.kb_per_split = p.kb_per_split;
-  args.lora_kb = 0;
-  args.lora_mod = 64;
-  args.partial = partial;
-  args.status = status;
-  // 96 KB of stages per CTA so that two CTAs share an SM.
-  constexpr int kStages = BN <= 64 ? 4 : 3;
-  return launch_gemm<kBM, BN, kStages, A_MN, BK_KIND, false, kEpiPartial>(dim3(1, p.tiles, p.splits), a, b, a, b,
-                                                                          args, stream);
-}
-
-template <bool A_MN, int BK_KIND>
-static cudaError_t dispatch_bn(int bn, const SkinnyPlan& p, const CUtensorMap& a, const CUtensorMap& b, int64_t red,
-                               float* partial, int* status, cudaStream_t stream) {
-  switch (bn) {
-    case 64: return launch_skinny_bn<64, A_MN, BK_KIND>(p, a, b, red, partial, status, stream);
-    case 128: return launch_skinny_bn<128, A_MN, BK_KIND>(p, a, b, red, partial, status, stream);
-    case 256: return launch_skinny_bn<256, A_MN, BK_KIND>(p, a, b, red, partial, status, stream);
-    default: return cudaErrorInvalidValue;
-  }
-}
-
-cudaError_t launch_skinny(SkinnyKind kind, const uint16_t* P0, const uint16_t* P1, int64_t M, int64_t K, int64_t N,
-                          int r, float scale, SkinnyOut out, float* partial, int* status, cudaStream_t stream) {
-  const SkinnyPlan p = plan_skinny(kind, M, K, N, r);
-  const int rp = lora_pad(r);
-  const int64_t pair_stride = static_cast<int64_t>(rp) * 4;  // bytes per row of a [rows x 2rp] bf16 pair
-  CUtensorMap ma, mb;
-  cudaError_t e;
-  int64_t rows, red;
-  const uint32_t bn = static_cast<uint32_t>(p.bn);
-  switch (kind) {
-    case SkinnyKind::kXA:  // A = X [M,K] K-major; B = A_lora [K,r] MN-major
-      rows = M;
-      red = K;
-      if (!make_map_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, P0, K, M, K * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
-          !make_map_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, P1, r, K, static_cast<int64_t>(r) * 2, 64, 64,
-                       CU_TENSOR_MAP_SWIZZLE_128B))
-        return cudaErrorInvalidValue;
-      e = dispatch_bn<false, kBTmaMN>(p.bn, p, ma, mb, red, partial, status, stream);
-      break;
-    case SkinnyKind::kDyBt:  // A = dY [M,N] K-major; B = B_lora [r,N] K-major
-      rows = M;
-      red = N;
-      if (!make_map_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, P0, N, M, N * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
-          !make_map_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, P1, N, r, N * 2, 64, bn, CU_TENSOR_MAP_SWIZZLE_128B))
-        return cudaErrorInvalidValue;
-      e = dispatch_bn<false, kBTmaK>(p.bn, p, ma, mb, red, partial, status, stream);
-      break;
-    case SkinnyKind::kTtDy:  // A = dY^T (dY [M,N]) MN-major; B = T pair [M,2rp] MN-major
-      rows = N;
-      red = M;
-      if (!make_map_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, P0, N, M, N * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-          !make_map_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, P1, 2 * rp, M, pair_stride, 64, 64,
-                       CU_TENSOR_MAP_SWIZZLE_128B))
-        return cudaErrorInvalidValue;
-      e = dispatch_bn<true, kBTmaMN>(p.bn, p, ma, mb, red, partial, status, stream);
-      break;
-    default:  // kXtU: A = X^T (X [M,K]) MN-major; B = U pair [M,2rp] MN-major
-      rows = K;
-      red = M;
-      if (!make_map_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, P0, K, M, K * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-          !make_map_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, P1, 2 * rp, M, pair_stride, 64, 64,
-                       CU_TENSOR_MAP_SWIZZLE_128B))
-        return cudaErrorInvalidValue;
-      e = dispatch_bn<true, kBTmaMN>(p.bn, p, ma, mb, red, partial, status, stream);
-      break;
-  }
-  if (e != cudaSuccess) return e;
-  const bool producer = kind == SkinnyKind::kXA || kind == SkinnyKind::kDyBt;
-  const int64_t rows_pad = static_cast<int64_t>(p.tiles) * kBM;
-  if (kind == SkinnyKind::kTtDy) {
-    const size_t smem = static_cast<size_t>(32) * (r + 1) * sizeof(float);
-    skinny_reduce_t_kernel<<<static_cast<unsigned>(ceil_div(rows, 32)), 256, smem, stream>>>(
-        partial, p.splits, rows_pad, p.bn, rows, r, rp, out.f32);
-  } else {
-    const int64_t n_out = rows * ((producer ? rp : r) / 4);
-    const int threads = 256;
-    skinny_reduce_kernel<<<static_cast<unsigned>(ceil_div(n_out, threads)), threads, 0, stream>>>(
-        partial, p.splits, rows_pad, p.bn, rows, r, rp, scale, static_cast<int>(kind), out.f32, out.pair);
-  }
-  return cudaGetLastError();
-}
-
-cudaError_t launch_split_pair(const float* v, int64_t rows, int r, uint16_t* pair, cudaStream_t stream) {
-  const int rp = lora_pad(r);
-  const int64_t n = rows * rp;
-  split_pair_kernel<<<static_cast<unsigned>(ceil_div(n, 256)), 256, 0, stream>>>(v, rows, r, rp, pair);
-  return cudaGetLastError();
 }
 
 }  // namespace qlora

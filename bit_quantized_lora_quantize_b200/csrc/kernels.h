@@ -32,7 +32,8 @@ cudaError_t launch_fused_dx(const uint16_t* dY, const uint8_t* codes, const uint
                             const float* absmax_scale, const uint16_t* Upair, const uint16_t* A, int64_t M, int64_t K,
                             int64_t N, int r, uint16_t* dX, int* status, const Nf4Params& P, cudaStream_t stream);
 
-// Skinny rank-r products (split over the reduction, deterministic reduction):
+// Rank-r products (reduction split over the CTAs of a cluster, partial tiles
+// summed in rank order through distributed shared memory):
 //   kXA   T  = s * X A          [M, r]   -> f32 (may be null) and pair
 //   kDyBt U  = s * dY B^T       [M, r]   -> f32 (may be null) and pair
 //   kTtDy dB = T^T dY  (fp32)   [r, N]   P1 = T pair
@@ -40,11 +41,11 @@ cudaError_t launch_fused_dx(const uint16_t* dY, const uint8_t* codes, const uint
 enum class SkinnyKind { kXA, kDyBt, kTtDy, kXtU };
 
 struct SkinnyPlan {
-  int tiles;        // 128-row output tiles
-  int splits;       // reduction splits
-  int kb_per_split; // 64-wide reduction blocks per split
-  int bn;           // output columns of the product (rp or 2*rp)
-  size_t partial_bytes;
+  int tiles;   // 128-row output tiles
+  int nkb;     // 64-deep reduction blocks
+  int kps;     // blocks per split
+  int splits;  // CTAs (one cluster) per tile
+  int bn;      // accumulator columns (rp for T and U, 2rp for dA, dB)
 };
 
 struct SkinnyOut {
@@ -55,11 +56,9 @@ struct SkinnyOut {
 SkinnyPlan plan_skinny(SkinnyKind kind, int64_t M, int64_t K, int64_t N, int r);
 
 cudaError_t launch_skinny(SkinnyKind kind, const uint16_t* P0, const uint16_t* P1, int64_t M, int64_t K, int64_t N,
-                          int r, float scale, SkinnyOut out, float* partial, int* status, cudaStream_t stream);
+                          int r, float scale, SkinnyOut out, int* status, cudaStream_t stream);
 
 // Pair matrix of a float32 [rows x r] matrix.
 cudaError_t launch_split_pair(const float* v, int64_t rows, int r, uint16_t* pair, cudaStream_t stream);
-
-size_t skinny_partial_bytes_max(int64_t M, int64_t K, int64_t N, int r);
 
 }  // namespace qlora

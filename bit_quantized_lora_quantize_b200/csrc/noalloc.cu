@@ -80,10 +80,9 @@ extern "C" qlora_status qlora_linear_fwd_noalloc(const uint16_t* X, int64_t M, i
                         reinterpret_cast<uintptr_t>(Y) | reinterpret_cast<uintptr_t>(T_save);
   if ((mis & 15u) || (reinterpret_cast<uintptr_t>(absmax_scale) & 3u)) return QLORA_ERR_ALIGNMENT;
 
-  // Scratch layout: [status word][T pair: bf16 M x 2rp][split partials of T].
+  // Scratch layout: [status word][T pair: bf16 M x 2rp].
   const size_t pair_bytes = round_up256(static_cast<size_t>(M) * 2 * lora_pad(r) * 2);
-  const size_t part_bytes = round_up256(plan_skinny(SkinnyKind::kXA, M, K, N, r).partial_bytes);
-  if (kStatusBytes + pair_bytes + part_bytes > kNoAllocScratchBytes) return QLORA_ERR_WORKSPACE;
+  if (kStatusBytes + pair_bytes > kNoAllocScratchBytes) return QLORA_ERR_WORKSPACE;
 
   void* base = nullptr;
   cudaError_t e = scratch_address(&base);
@@ -91,12 +90,12 @@ extern "C" qlora_status qlora_linear_fwd_noalloc(const uint16_t* X, int64_t M, i
   unsigned char* ws = static_cast<unsigned char*>(base);
   int* status = reinterpret_cast<int*>(ws);
   uint16_t* Tpair = reinterpret_cast<uint16_t*>(ws + kStatusBytes);
-  float* partial = reinterpret_cast<float*>(ws + kStatusBytes + pair_bytes);
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
 
-  e = cudaMemsetAsync(status, 0, sizeof(int), st);
+  // Clear the status word: a call that timed out earlier may have left it set.
+  e = cudaMemsetAsync(ws, 0, sizeof(int), st);
   if (e == cudaSuccess)
-    e = launch_skinny(SkinnyKind::kXA, X, A, M, K, N, r, scale, SkinnyOut{T_save, Tpair}, partial, status, st);
+    e = launch_skinny(SkinnyKind::kXA, X, A, M, K, N, r, scale, SkinnyOut{T_save, Tpair}, status, st);
   if (e == cudaSuccess)
     e = launch_fused_fwd(X, codes, absmax_q, absmax_scale, Tpair, B, M, K, N, r, Y, status, nf4_params(), st);
   return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;

@@ -158,9 +158,10 @@ QLORA_API qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, c
  *   qlora_linear_fwd, minus workspace/ws_bytes.  The call allocates nothing:
  *   its scratch is one fixed 16 MiB device array inside this library, which
  *   every GPU that loads the library keeps until the process exits.
- *   - Shapes whose forward scratch (status word + bf16 pair of T + split
- *     partials of T) exceeds 16 MiB return QLORA_ERR_WORKSPACE and launch
- *     nothing; the 4096 x 4096, 4096-token, r = 64 layer needs about 11.5 MiB.
+ *   - Shapes whose forward scratch (status word + bf16 pair of T, i.e.
+ *     256 + 4*M*rp bytes with rp = r rounded up to 64) exceeds 16 MiB return
+ *     QLORA_ERR_WORKSPACE and launch nothing; 4096 tokens at r = 64 need
+ *     1 MiB, so up to 32768 tokens fit at r <= 64.
  *   - The first call on a device (with that device current, and `stream`
  *     belonging to it) looks up the array's device address once; make that
  *     first call before any stream capture on that device.
