@@ -52,6 +52,7 @@ struct GemmArgs {
   const float* absmax_scale;
   int64_t w_rows;  // N of the packed weight [N, K]
   int64_t w_cols;  // K
+  int abs_tma;     // dX: the stage's 8-bit constant codes arrive by TMA (K % 1024 == 0)
   int lora_mod;    // padded rank rp: LoRA stage lk reads the adapter at (64*lk) mod rp
   int* status;
   Nf4Params nf4;
@@ -66,7 +67,10 @@ struct SmemLayout {
   static constexpr int kA = 0;
   static constexpr int kB = kA + STAGES * kABytes;
   static constexpr int kC = kB + STAGES * kBBytes;
-  static constexpr int kBar = kC + STAGES * kCBytes;
+  static constexpr int kLvl2 = kC + STAGES * kCBytes;            // fp32(k/255), 256 floats
+  static constexpr int kAbs = kLvl2 + (kDecode ? 1024 : 0);       // 8-bit constant codes (dX)
+  static constexpr int kAbsBytes = (BK_KIND == kBNf4MN) ? 1024 : 0;
+  static constexpr int kBar = kAbs + STAGES * kAbsBytes;
   static constexpr int kNumBars = 3 * STAGES + 1;
   static constexpr int kTmemSlot = kBar + kNumBars * 8;
   static constexpr int kAbort = kTmemSlot + 4;
@@ -88,7 +92,7 @@ template <int BM, int BN, int STAGES, bool A_MN, int BK_KIND, bool B2_MN, int EP
 __global__ void __launch_bounds__((BK_KIND == kBNf4K || BK_KIND == kBNf4MN) ? 384 : 256, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
-                const GemmArgs args) {
+                const __grid_constant__ CUtensorMap tmAbs, const GemmArgs args) {
   using L = SmemLayout<BM, BN, STAGES, BK_KIND>;
   constexpr bool kDecode = L::kDecode;
   constexpr bool kBMN = (BK_KIND == kBTmaMN || BK_KIND == kBNf4MN);
@@ -105,6 +109,8 @@ __global__ void __launch_bounds__((BK_KIND == kBNf4K || BK_KIND == kBNf4MN) ? 38
   uint8_t* sA = smem + L::kA;
   uint8_t* sB = smem + L::kB;
   uint8_t* sC = smem + L::kC;
+  float* lvl2 = reinterpret_cast<float*>(smem + L::kLvl2);
+  uint8_t* sAbs = smem + L::kAbs;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBar);
   uint64_t* empty = full + STAGES;
   uint64_t* decoded = empty + STAGES;
@@ -162,7 +168,8 @@ __global__ void __launch_bounds__((BK_KIND == kBNf4K || BK_KIND == kBNf4MN) ? 38
         uint8_t* b_dst = sB + s * L::kBBytes;
         if (i < num_kb) {
           const int kb = kb_begin + i;
-          mbar_arrive_expect_tx(&full[s], kABytes + (kDecode ? kCodeBytes : L::kBBytes));
+          const bool abs_tma = (BK_KIND == kBNf4MN) && args.abs_tma;
+          mbar_arrive_expect_tx(&full[s], kABytes + (kDecode ? kCodeBytes : L::kBBytes) + (abs_tma ? 1024 : 0));
           if (!A_MN) {
             tma_load_2d(&tmA, &full[s], a_dst, kb * kBK, tile_m * BM);
           } else {
@@ -180,6 +187,9 @@ __global__ void __launch_bounds__((BK_KIND == kBNf4K || BK_KIND == kBNf4MN) ? 38
           } else {
             // codes: 64 rows (reduction) x 128 bytes (256 outputs)
             tma_load_2d(&tmB, &full[s], sC + s * kCodeBytes, tile_n * 128, kb * kBK);
+            // 8-bit constant codes of those 64 rows: a 16-byte-wide box that
+            // starts at the 16-aligned block column at or before tile_n * 4
+            if (abs_tma) tma_load_2d(&tmAbs, &full[s], sAbs + s * 1024, (tile_n * 4) & ~15, kb * kBK);
           }
         } else {
           // LoRA stage: [T_hi | T_lo] (or U) against the adapter, which is read
@@ -253,6 +263,8 @@ __global__ void __launch_bounds__((BK_KIND == kBNf4K || BK_KIND == kBNf4MN) ? 38
       const WaitCtx ctx{abort_flag, args.status, 3};
       const int d = threadIdx.x - 128;  // 0..255
       const int64_t blocks_per_row = args.w_cols / 64;
+      lvl2[d] = level2_value(d);
+      asm volatile("bar.sync 1, 256;" ::: "memory");  // decoder warps only
       if (BK_KIND == kBNf4K) {
         // Thread d decodes weight row n = tile_n*256 + d, one 64-wide block per stage.
         const int64_t n = static_cast<int64_t>(tile_n) * 256 + d;
@@ -283,7 +295,7 @@ __global__ void __launch_bounds__((BK_KIND == kBNf4K || BK_KIND == kBNf4MN) ? 38
             const uint4 v0 = lds128(src);
             const uint4 v1 = lds128(src + 16);
             const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-            const Nf4Lut lut = make_lut(args.nf4, block_constant(q2, c1));
+            const Nf4Lut lut = make_lut(args.nf4, __fmul_rn(lvl2[q2], c1));
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
               uint32_t o[4];
@@ -309,11 +321,13 @@ __global__ void __launch_bounds__((BK_KIND == kBNf4K || BK_KIND == kBNf4MN) ? 38
         const bool col_ok = kob < blocks_per_row;
         const uint32_t b_off = j * 8192 + (nl >> 3) * 1024;
         const int r8 = nl & 7;
+        const bool abs_tma = args.abs_tma != 0;
+        const int abs_col = static_cast<int>(kob - ((static_cast<int64_t>(tile_n) * 4) & ~int64_t(15)));
         auto load_const = [&](int i, uint32_t& q, float& c) {
           const int64_t n = static_cast<int64_t>(kb_begin + i) * 64 + nl;
           if (col_ok && n < args.w_rows) {
             const int64_t b = n * blocks_per_row + kob;
-            q = __ldg(args.absmax_q + b);
+            q = abs_tma ? 0u : __ldg(args.absmax_q + b);
             c = __ldg(args.absmax_scale + (b >> 8));
             return true;
           }
@@ -337,7 +351,8 @@ __global__ void __launch_bounds__((BK_KIND == kBNf4K || BK_KIND == kBNf4MN) ? 38
             const uint4 v0 = lds128(row + (((2 * j) ^ r8) << 4));
             const uint4 v1 = lds128(row + (((2 * j + 1) ^ r8) << 4));
             const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-            const Nf4Lut lut = make_lut(args.nf4, block_constant(q2, c1));
+            if (abs_tma) q2 = sAbs[s * 1024 + nl * 16 + abs_col];
+            const Nf4Lut lut = make_lut(args.nf4, __fmul_rn(lvl2[q2], c1));
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
               uint32_t o[4];
@@ -411,14 +426,15 @@ __global__ void __launch_bounds__((BK_KIND == kBNf4K || BK_KIND == kBNf4MN) ? 38
 // ----------------------------------------------------------------- host side
 template <int BM, int BN, int STAGES, bool A_MN, int BK_KIND, bool B2_MN, int EPI>
 static cudaError_t launch_gemm(dim3 grid, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& a2,
-                               const CUtensorMap& b2, const GemmArgs& args, cudaStream_t stream) {
+                               const CUtensorMap& b2, const CUtensorMap& abs, const GemmArgs& args,
+                               cudaStream_t stream) {
   using L = SmemLayout<BM, BN, STAGES, BK_KIND>;
   auto kern = gemm_kernel<BM, BN, STAGES, A_MN, BK_KIND, B2_MN, EPI>;
   static_assert(L::kDynamic <= 232448, "shared memory budget");
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kDynamic);
   if (e != cudaSuccess) return e;
   const int threads = L::kDecode ? 384 : 256;
-  kern<<<grid, threads, L::kDynamic, stream>>>(a, b, a2, b2, args);
+  kern<<<grid, threads, L::kDynamic, stream>>>(a, b, a2, b2, abs, args);
   return cudaGetLastError();
 }
 
@@ -452,7 +468,8 @@ cudaError_t launch_fused_fwd(const uint16_t* X, const uint8_t* codes, const uint
   args.status = status;
   args.nf4 = P;
   dim3 grid(static_cast<unsigned>((N + 255) / 256), static_cast<unsigned>((M + kFusedBM - 1) / kFusedBM), 1);
-  return launch_gemm<kFusedBM, 256, kFusedStages, false, kBNf4K, true, kEpiBf16>(grid, mX, mC, mT, mB, args, stream);
+  return launch_gemm<kFusedBM, 256, kFusedStages, false, kBNf4K, true, kEpiBf16>(grid, mX, mC, mT, mB, mB, args,
+                                                                                   stream);
 }
 
 cudaError_t launch_fused_dx(const uint16_t* dY, const uint8_t* codes, const uint8_t* absmax_q,
@@ -467,7 +484,14 @@ cudaError_t launch_fused_dx(const uint16_t* dY, const uint8_t* codes, const uint
       !make_map_2d(&mA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, r, K, static_cast<int64_t>(r) * 2, 64, 256,
                    CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
+  // The 8-bit constant codes as a [N x K/64] byte matrix; rows must be a
+  // multiple of 16 bytes for TMA, i.e. K % 1024 == 0 (otherwise plain loads).
+  CUtensorMap mAbs = mA;
+  const bool abs_tma = (K % 1024 == 0) &&
+                       make_map_2d(&mAbs, CU_TENSOR_MAP_DATA_TYPE_UINT8, absmax_q, K / 64, N, K / 64, 16, 64,
+                                   CU_TENSOR_MAP_SWIZZLE_NONE);
   GemmArgs args{};
+  args.abs_tma = abs_tma ? 1 : 0;
   args.nkb_total = static_cast<int>((N + 63) / 64);
   args.kb_per_split = args.nkb_total;
   args.lora_kb = 2 * rp / 64;
@@ -483,7 +507,7 @@ cudaError_t launch_fused_dx(const uint16_t* dY, const uint8_t* codes, const uint
   args.status = status;
   args.nf4 = P;
   dim3 grid(static_cast<unsigned>((K + 255) / 256), static_cast<unsigned>((M + kFusedBM - 1) / kFusedBM), 1);
-  return launch_gemm<kFusedBM, 256, kFusedStages, false, kBNf4MN, false, kEpiBf16>(grid, mD, mC, mU, mA, args,
+  return launch_gemm<kFusedBM, 256, kFusedStages, false, kBNf4MN, false, kEpiBf16>(grid, mD, mC, mU, mA, mAbs, args,
                                                                                     stream);
 }
 
