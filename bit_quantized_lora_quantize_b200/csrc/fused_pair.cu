@@ -1,0 +1,538 @@
+// Fused NF4 dequant-GEMMs on CTA pairs (tcgen05 cta_group::2), sm_100a.
+//
+// "AI Glossary: QLoRA", second paragraph, and "QLoRA's Working Process":
+// the frozen 4-bit weight is turned back into BFloat16 on the fly for each
+// product; no bf16 copy of W is stored.
+//
+//   forward         Y  = X  W'^T + [T_hi | T_lo] [B ; B]      (B operand K-major)
+//   input gradient  dX = dY W'   + [U_hi | U_lo] [A^T ; A^T]  (B operand MN-major)
+//
+// Two CTAs of a cluster compute one 512 x 256 output tile.  Each CTA holds
+// 2 x 128 rows of the activation tile (one 128-row half of each of two
+// M = 256 pair-MMAs) and decodes its own 128-row half of the weight tile; the
+// pair's tensor cores read both halves.  Every decoded weight therefore feeds
+// 512 output rows, which halves the decode work per tensor-core cycle
+// compared with a 256-row single-CTA tile, and a stage is 52 KB so four
+// stages fit.
+//
+// Per CTA: warp 0 issues TMA (activation rows and LoRA tiles signal the
+// leader CTA's barrier, packed codes a local one; no multicast loads), warp 1
+// allocates TMEM (both CTAs) and, in the leader only, issues the MMAs and
+// commits them to both CTAs' barriers; warps 4-7 decode the even stages and
+// warps 8-11 the odd ones (one 64-weight block per thread per stage), then
+// all eight drain the two 128 x 256 fp32 accumulators.
+#include <algorithm>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "kernels.h"
+#include "nf4_device.cuh"
+#include "ptx.cuh"
+#include "tensor_map.h"
+
+namespace qlora {
+
+namespace {
+
+constexpr int kPairRows = 512;    // output rows of a pair tile
+constexpr int kPairCols = 256;    // output columns of a pair tile
+constexpr int kDepth = 64;
+constexpr int kStages = 4;
+constexpr int kThreads = 384;
+constexpr int kDecWarps = 4;      // decoder warps per stage (warps 4-7 even stages, 8-11 odd)
+
+struct PairArgs {
+  int nkb;          // main 64-deep stages
+  int lora_kb;      // LoRA stages (hi and lo halves of the pair)
+  int lora_mod;     // rp: LoRA stage lk reads the adapter at (64*lk) mod rp
+  int rows, cols;   // output extent
+  int64_t ld_out;
+  uint16_t* out;
+  const uint8_t* absmax_q;
+  const float* absmax_scale;
+  int64_t w_rows, w_cols;  // N, K of the packed weight
+  int abs_tma;             // dX: 8-bit constant codes by TMA
+  int* status;
+  Nf4Params nf4;
+};
+
+template <bool MNB>
+struct PairSmem {
+  static constexpr int kA = 2 * 128 * kDepth * 2;   // 32 KB: two 128-row halves
+  static constexpr int kB = 128 * kDepth * 2;       // 16 KB: this CTA's half of the weight tile
+  static constexpr int kC = 4096;                   // packed codes of that half
+  static constexpr int kAbs = MNB ? 1024 : 0;
+  static constexpr int offA = 0;
+  static constexpr int offB = offA + kStages * kA;
+  static constexpr int offC = offB + kStages * kB;
+  static constexpr int offAbs = offC + kStages * kC;
+  static constexpr int offLvl2 = offAbs + kStages * kAbs;
+  static constexpr int offBar = offLvl2 + 1024;
+  // full, cfull, empty, decoded per stage; acc_full
+  static constexpr int kNumBars = 4 * kStages + 1;
+  static constexpr int offSlot = offBar + kNumBars * 8;
+  static constexpr int offAbort = offSlot + 4;
+  static constexpr int kTotal = offAbort + 4;
+  static constexpr int kDynamic = kTotal + 1024;
+};
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Shared::cluster address of the same object in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_rank(const void* p, uint32_t rank) {
+  uint32_t d;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(d) : "r"(smem_u32(p)), "r"(rank));
+  return d;
+}
+__device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap* map, uint32_t mbar_cluster, void* dst, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(mbar_cluster), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t mbar_cluster) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(mbar_cluster) : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void umma_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive on the barrier at this offset in both CTAs once the issued MMAs end.
+__device__ __forceinline__ void umma_commit_pair(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"(static_cast<uint16_t>(3))
+      : "memory");
+}
+
+template <bool MNB>
+__global__ void __launch_bounds__(kThreads, 1)
+    fused_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmC,
+                      const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
+                      const __grid_constant__ CUtensorMap tmAbs, const PairArgs args) {
+  using L = PairSmem<MNB>;
+  constexpr uint32_t kTmemCols = 512;  // two 128 x 256 fp32 accumulators
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem + L::offA;
+  uint8_t* sB = smem + L::offB;
+  uint8_t* sC = smem + L::offC;
+  uint8_t* sAbs = smem + L::offAbs;
+  float* lvl2 = reinterpret_cast<float*>(smem + L::offLvl2);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::offBar);  // leader: both CTAs' TMA bytes
+  uint64_t* cfull = full + kStages;                                // local: this CTA's codes
+  uint64_t* empty = cfull + kStages;                               // local: MMA done with the stage
+  uint64_t* decoded = empty + kStages;                             // leader: both CTAs' decoders
+  uint64_t* acc_full = decoded + kStages;                          // local: accumulators ready
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::offSlot);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::offAbort);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();  // 0 = leader
+  const int tile_n = blockIdx.x >> 1;
+  const int tile_m = blockIdx.y;
+  const int total = args.nkb + args.lora_kb;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&cfull[s], 1);
+      mbar_init(&empty[s], 1);
+      mbar_init(&decoded[s], 2 * kDecWarps);
+    }
+    mbar_init(acc_full, 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmC);
+    tma_prefetch_desc(&tmA2);
+    tma_prefetch_desc(&tmB2);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // the leader's barriers exist before the peer signals them
+  tc_fence_after();
+  const uint32_t tmem_acc = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const WaitCtx ctx{abort_flag, args.status, 21};
+      int issued = 0;
+      for (int i = 0; i < total; ++i) {
+        const int s = i % kStages;
+        const uint32_t ph = (i / kStages) & 1;
+        if (!mbar_wait(&empty[s], ph ^ 1, ctx)) break;
+        const uint32_t full_leader = map_rank(&full[s], 0);
+        uint8_t* a_dst = sA + s * L::kA;
+        uint8_t* b_dst = sB + s * L::kB;
+        const int row0 = tile_m * kPairRows + static_cast<int>(rank) * 128;
+        if (i < args.nkb) {
+          const int kb = i;
+          if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * L::kA);
+          tma_load_2d_pair(&tmA, full_leader, a_dst, kb * kDepth, row0);
+          tma_load_2d_pair(&tmA, full_leader, a_dst + 16384, kb * kDepth, row0 + 256);
+          const bool abs_tma = MNB && args.abs_tma;
+          mbar_arrive_expect_tx(&cfull[s], L::kC + (abs_tma ? 1024 : 0));
+          if (!MNB) {
+            // codes [N, K/2]: this CTA's 128 weight rows x 32 bytes
+            tma_load_2d(&tmC, &cfull[s], sC + s * L::kC, kb * 32, tile_n * kPairCols + static_cast<int>(rank) * 128);
+          } else {
+            // codes: 64 reduction rows x 64 bytes (this CTA's 128 outputs)
+            tma_load_2d(&tmC, &cfull[s], sC + s * L::kC, tile_n * 128 + static_cast<int>(rank) * 64, kb * kDepth);
+            if (abs_tma)
+              tma_load_2d(&tmAbs, &cfull[s], sAbs + s * 1024, ((tile_n * 4) + static_cast<int>(rank) * 2) & ~15,
+                          kb * kDepth);
+          }
+        } else {
+          const int lk = i - args.nkb;
+          const int lb = (lk * kDepth) % args.lora_mod;
+          if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * (L::kA + L::kB));
+          tma_load_2d_pair(&tmA2, full_leader, a_dst, lk * kDepth, row0);
+          tma_load_2d_pair(&tmA2, full_leader, a_dst + 16384, lk * kDepth, row0 + 256);
+          const int c0 = tile_n * kPairCols + static_cast<int>(rank) * 128;
+          if (!MNB) {
+            // LoRA B [r, N] (MN-major): this CTA's 128 output columns
+            tma_load_2d_pair(&tmB2, full_leader, b_dst, c0, lb);
+            tma_load_2d_pair(&tmB2, full_leader, b_dst + 8192, c0 + 64, lb);
+          } else {
+            // LoRA A [K, r] (K-major): this CTA's 128 output rows of A
+            tma_load_2d_pair(&tmB2, full_leader, b_dst, lb, c0);
+          }
+        }
+        ++issued;
+      }
+      if (*abort_flag) {
+        for (int i = (issued > kStages ? issued - kStages : 0); i < issued; ++i) {
+          const uint64_t t0 = globaltimer_ns();
+          const int s = i % kStages;
+          const uint32_t ph = (i / kStages) & 1;
+          while (globaltimer_ns() - t0 < kWaitTimeoutNs &&
+                 !(mbar_try_wait(&cfull[s], ph) && (rank != 0 || mbar_try_wait(&full[s], ph)))) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA (leader)
+    if (lane == 0 && rank == 0) {
+      const WaitCtx ctx{abort_flag, args.status, 22};
+      // M = 256 across the pair, N = 256 (each CTA supplies 128 columns of B).
+      const uint32_t idesc_main = idesc_bf16_f32(256, 256, false, MNB);
+      const uint32_t idesc_lora = idesc_bf16_f32(256, 256, false, !MNB);
+      bool ok = true;
+      for (int i = 0; i < total && ok; ++i) {
+        const int s = i % kStages;
+        const uint32_t ph = (i / kStages) & 1;
+        const bool main_stage = i < args.nkb;
+        if (!mbar_wait(&full[s], ph, ctx)) { ok = false; break; }
+        if (main_stage && !mbar_wait(&decoded[s], ph, ctx)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t a_base = smem_u32(sA + s * L::kA);
+        const uint32_t b_base = smem_u32(sB + s * L::kB);
+        const bool b_mn = main_stage ? MNB : !MNB;
+#pragma unroll
+        for (int kk = 0; kk < kDepth / 16; ++kk) {
+          const uint64_t bdesc = b_mn ? smem_desc_sw128(b_base + kk * 2048, 8192, 1024)
+                                      : smem_desc_sw128(b_base + kk * 32, 16, 1024);
+          const uint32_t idesc = main_stage ? idesc_main : idesc_lora;
+          const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+          umma_pair(tmem_acc, smem_desc_sw128(a_base + kk * 32, 16, 1024), bdesc, idesc, acc);
+          umma_pair(tmem_acc + 256, smem_desc_sw128(a_base + 16384 + kk * 32, 16, 1024), bdesc, idesc, acc);
+        }
+        umma_commit_pair(&empty[s]);
+      }
+      if (ok) umma_commit_pair(acc_full);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ decoders (warps 4-11)
+    // Two groups of four warps take alternate stages; in each group thread d
+    // decodes one 64-weight block of this CTA's half of the weight tile.
+    {
+      const WaitCtx ctx{abort_flag, args.status, 23};
+      const int grp = (warp - 4) >> 2;          // 0: even stages, 1: odd stages
+      const int d = (threadIdx.x - 128) & 127;  // 0..127
+      lvl2[threadIdx.x - 128] = level2_value(threadIdx.x - 128);
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      const int64_t blocks_per_row = args.w_cols / 64;
+      if (!MNB) {
+        // Thread d decodes weight row n (this CTA's half), one block per stage.
+        const int64_t n = static_cast<int64_t>(tile_n) * kPairCols + rank * 128 + d;
+        const bool row_ok = n < args.w_rows;
+        const uint32_t b_row = (d >> 3) * 1024;
+        const int r8 = d & 7;
+        int64_t blk = n * blocks_per_row + grp;
+        uint32_t q2 = 0;
+        float c1 = 0.0f;
+        if (row_ok && grp < args.nkb) {
+          q2 = __ldg(args.absmax_q + blk);
+          c1 = __ldg(args.absmax_scale + (blk >> 8));
+        }
+        for (int i = grp; i < args.nkb; i += 2) {
+          const int s = i % kStages;
+          const uint32_t ph = (i / kStages) & 1;
+          uint32_t q2n = 0;
+          float c1n = 0.0f;
+          if (row_ok && i + 2 < args.nkb) {
+            q2n = __ldg(args.absmax_q + blk + 2);
+            c1n = __ldg(args.absmax_scale + ((blk + 2) >> 8));
+          }
+          if (!__all_sync(0xFFFFFFFFu, mbar_wait(&cfull[s], ph, ctx))) break;
+          uint8_t* dst = sB + s * L::kB + b_row;
+          if (row_ok) {
+            // 32-byte rows with the 32-byte swizzle: chunk c at c ^ ((d >> 2) & 1)
+            const uint8_t* src = sC + s * L::kC + d * 32;
+            const int sw = (d >> 2) & 1;
+            const uint4 v0 = *reinterpret_cast<const uint4*>(src + ((0 ^ sw) << 4));
+            const uint4 v1 = *reinterpret_cast<const uint4*>(src + ((1 ^ sw) << 4));
+            const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+            const Nf4Lut lut = make_lut(args.nf4, __fmul_rn(lvl2[q2], c1));
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              uint32_t o[4];
+              decode8(lut, w[c], o);
+              *reinterpret_cast<uint4*>(dst + sw128_offset(r8, c)) = make_uint4(o[0], o[1], o[2], o[3]);
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(dst + sw128_offset(r8, c)) = make_uint4(0, 0, 0, 0);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(map_rank(&decoded[s], 0));
+          q2 = q2n;
+          c1 = c1n;
+          blk += 2;
+        }
+      } else {
+        // Thread d: reduction row nl of the stage, output atom j (64 outputs).
+        const int nl = d & 63;
+        const int j = d >> 6;  // 0..1
+        const int64_t kob = static_cast<int64_t>(tile_n) * 4 + rank * 2 + j;  // 64-wide output block
+        const bool col_ok = kob < blocks_per_row;
+        const uint32_t b_off = j * 8192 + (nl >> 3) * 1024;
+        const int r8 = nl & 7;
+        const bool abs_tma = args.abs_tma != 0;
+        const int abs_col = static_cast<int>(kob - ((static_cast<int64_t>(tile_n) * 4 + rank * 2) & ~int64_t(15)));
+        auto load_const = [&](int i, uint32_t& q, float& c) {
+          const int64_t n = static_cast<int64_t>(i) * 64 + nl;
+          if (col_ok && n < args.w_rows) {
+            const int64_t b = n * blocks_per_row + kob;
+            q = abs_tma ? 0u : __ldg(args.absmax_q + b);
+            c = __ldg(args.absmax_scale + (b >> 8));
+            return true;
+          }
+          q = 0;
+          c = 0.0f;
+          return false;
+        };
+        uint32_t q2 = 0;
+        float c1 = 0.0f;
+        bool ok_cur = grp < args.nkb ? load_const(grp, q2, c1) : false;
+        for (int i = grp; i < args.nkb; i += 2) {
+          const int s = i % kStages;
+          const uint32_t ph = (i / kStages) & 1;
+          uint32_t q2n = 0;
+          float c1n = 0.0f;
+          const bool ok_next = (i + 2 < args.nkb) ? load_const(i + 2, q2n, c1n) : false;
+          if (!__all_sync(0xFFFFFFFFu, mbar_wait(&cfull[s], ph, ctx))) break;
+          uint8_t* dst = sB + s * L::kB + b_off;
+          if (ok_cur) {
+            // 64-byte rows with the 64-byte swizzle: chunk c at c ^ ((nl >> 1) & 3)
+            const uint8_t* row = sC + s * L::kC + nl * 64;
+            const int sw = (nl >> 1) & 3;
+            const uint4 v0 = *reinterpret_cast<const uint4*>(row + (((2 * j) ^ sw) << 4));
+            const uint4 v1 = *reinterpret_cast<const uint4*>(row + (((2 * j + 1) ^ sw) << 4));
+            const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+            if (abs_tma) q2 = sAbs[s * 1024 + nl * 16 + abs_col];
+            const Nf4Lut lut = make_lut(args.nf4, __fmul_rn(lvl2[q2], c1));
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              uint32_t o[4];
+              decode8(lut, w[c], o);
+              *reinterpret_cast<uint4*>(dst + sw128_offset(r8, c)) = make_uint4(o[0], o[1], o[2], o[3]);
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(dst + sw128_offset(r8, c)) = make_uint4(0, 0, 0, 0);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(map_rank(&decoded[s], 0));
+          q2 = q2n;
+          c1 = c1n;
+          ok_cur = ok_next;
+        }
+      }
+    }
+    // ------------------------------------------------------------ epilogue (warps 4-11)
+    {
+      const WaitCtx ctx{abort_flag, args.status, 24};
+      const int q = warp & 3;
+      const int h = (warp - 4) >> 2;  // accumulator (first or second M = 256 MMA)
+      const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(acc_full, 0, ctx));
+      tc_fence_after();
+      if (ok) {
+        const int row = tile_m * kPairRows + h * 256 + static_cast<int>(rank) * 128 + q * 32 + lane;
+        const uint32_t t_row = tmem_acc + (static_cast<uint32_t>(q * 32) << 16) + h * 256;
+#pragma unroll 1
+        for (int cc = 0; cc < kPairCols / 32; ++cc) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(t_row + cc * 32, v);
+          tmem_wait_ld();
+          const int col0 = tile_n * kPairCols + cc * 32;
+          if (row < args.rows) {
+            uint16_t* out = args.out + static_cast<int64_t>(row) * args.ld_out;
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              const int col = col0 + g * 8;
+              if (col < args.cols) {
+                uint32_t p[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                  p[e] = pack_bf16x2_rn(__uint_as_float(v[g * 8 + 2 * e]), __uint_as_float(v[g * 8 + 2 * e + 1]));
+                *reinterpret_cast<uint4*>(out + col) = make_uint4(p[0], p[1], p[2], p[3]);
+              }
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // neither CTA leaves while the pair's MMAs or signals may touch it
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_acc, kTmemCols);
+  }
+}
+
+template <bool MNB>
+cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& c, const CUtensorMap& a2, const CUtensorMap& b2,
+                        const CUtensorMap& abs, const PairArgs& args, int tiles_n, int tiles_m, cudaStream_t stream) {
+  using L = PairSmem<MNB>;
+  static_assert(L::kDynamic <= 232448, "shared memory budget");
+  auto kern = fused_pair_kernel<MNB>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kDynamic);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * tiles_n), static_cast<unsigned>(tiles_m), 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = L::kDynamic;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a, c, a2, b2, abs, args);
+}
+
+}  // namespace
+
+cudaError_t launch_fused_fwd(const uint16_t* X, const uint8_t* codes, const uint8_t* absmax_q,
+                             const float* absmax_scale, const uint16_t* Tpair, const uint16_t* B, int64_t M, int64_t K,
+                             int64_t N, int r, uint16_t* Y, int* status, const Nf4Params& P, cudaStream_t stream) {
+  const int rp = lora_pad(r);
+  CUtensorMap mX, mC, mT, mB;
+  if (!make_map_2d(&mX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, K * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&mC, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, K / 2, N, K / 2, 32, 128, CU_TENSOR_MAP_SWIZZLE_32B) ||
+      !make_map_2d(&mT, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Tpair, 2 * rp, M, static_cast<int64_t>(rp) * 4, 64, 128,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&mB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, B, N, r, N * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  PairArgs args{};
+  args.nkb = static_cast<int>(K / 64);
+  args.lora_kb = 2 * rp / 64;
+  args.lora_mod = rp;
+  args.rows = static_cast<int>(M);
+  args.cols = static_cast<int>(N);
+  args.ld_out = N;
+  args.out = Y;
+  args.absmax_q = absmax_q;
+  args.absmax_scale = absmax_scale;
+  args.w_rows = N;
+  args.w_cols = K;
+  args.abs_tma = 0;
+  args.status = status;
+  args.nf4 = P;
+  const int tiles_n = static_cast<int>((N + kPairCols - 1) / kPairCols);
+  const int tiles_m = static_cast<int>((M + kPairRows - 1) / kPairRows);
+  return launch_pair<false>(mX, mC, mT, mB, mB, args, tiles_n, tiles_m, stream);
+}
+
+cudaError_t launch_fused_dx(const uint16_t* dY, const uint8_t* codes, const uint8_t* absmax_q,
+                            const float* absmax_scale, const uint16_t* Upair, const uint16_t* A, int64_t M, int64_t K,
+                            int64_t N, int r, uint16_t* dX, int* status, const Nf4Params& P, cudaStream_t stream) {
+  const int rp = lora_pad(r);
+  CUtensorMap mD, mC, mU, mA;
+  if (!make_map_2d(&mD, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dY, N, M, N * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&mC, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, K / 2, N, K / 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !make_map_2d(&mU, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Upair, 2 * rp, M, static_cast<int64_t>(rp) * 4, 64, 128,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&mA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, r, K, static_cast<int64_t>(r) * 2, 64, 128,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  CUtensorMap mAbs = mA;
+  const bool abs_tma = (K % 1024 == 0) &&
+                       make_map_2d(&mAbs, CU_TENSOR_MAP_DATA_TYPE_UINT8, absmax_q, K / 64, N, K / 64, 16, 64,
+                                   CU_TENSOR_MAP_SWIZZLE_NONE);
+  PairArgs args{};
+  args.nkb = static_cast<int>((N + 63) / 64);
+  args.lora_kb = 2 * rp / 64;
+  args.lora_mod = rp;
+  args.rows = static_cast<int>(M);
+  args.cols = static_cast<int>(K);
+  args.ld_out = K;
+  args.out = dX;
+  args.absmax_q = absmax_q;
+  args.absmax_scale = absmax_scale;
+  args.w_rows = N;
+  args.w_cols = K;
+  args.abs_tma = abs_tma ? 1 : 0;
+  args.status = status;
+  args.nf4 = P;
+  const int tiles_n = static_cast<int>((K + kPairCols - 1) / kPairCols);
+  const int tiles_m = static_cast<int>((M + kPairRows - 1) / kPairRows);
+  return launch_pair<true>(mD, mC, mU, mA, mAbs, args, tiles_n, tiles_m, stream);
+}
+
+}  // namespace qlora
