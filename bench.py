@@ -172,6 +172,41 @@ def traffic_for(kernel: str):
         return None
 
 
+def small_m_sweep(q, synthetic, dev, flush, iters=10):
+    """Small-M forward (W [N x 8192] NF4, M tokens, r = 64): NF4 weight bytes
+    streamed per second, L2 flushed before every timed call."""
+    import torch
+
+    peaks = load_peaks()
+    out = []
+    for N in (8192, 22016):
+        W = synthetic.weight_only(N, 8192, seed=4).to(dev)
+        Wp = q.qlora_quantize_nf4(W)
+        del W
+        nf4_bytes = Wp.codes.numel() + Wp.absmax_q.numel() + 4 * Wp.absmax_scale.numel()
+        for M in (1, 4, 16, 64):
+            case = synthetic.small_m_case(M, N)
+            X, A, B = (t.to(dev) for t in (case.X, case.A, case.B))
+            ws = q.new_workspace(M, 8192, N, 64, dev)
+            Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+            T = torch.empty(M, 64, dtype=torch.float32, device=dev)
+            for _ in range(3):
+                q.qlora_linear_fwd(X, Wp, A, B, 0.25, workspace=ws, Y=Y, T_save=T)
+            stream = torch.cuda.current_stream()
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(iters)]
+            for i in range(iters):
+                flush.zero_()
+                evs[i][0].record(stream)
+                q.qlora_linear_fwd(X, Wp, A, B, 0.25, workspace=ws, Y=Y, T_save=T)
+                evs[i][1].record(stream)
+            torch.cuda.synchronize()
+            us = sorted(a.elapsed_time(b) * 1e3 for a, b in evs)[iters // 2]
+            gbs = nf4_bytes / (us * 1e-6) / 1e9
+            out.append({"N": N, "K": 8192, "M": M, "us": us, "nf4_weight_gbs": gbs,
+                        "frac_hbm": gbs / peaks["hbm_gbs"], "nf4_bytes": nf4_bytes})
+    return out
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -275,6 +310,8 @@ def run_ours(args, rank, world, local_rank):
     if q.qlora_check_status(ws) != 0:
         raise RuntimeError("device pipeline timeout during timing")
 
+    small_m = small_m_sweep(q, synthetic, dev, flush) if (rank == 0 and not args.no_small_m) else None
+
     if rank != 0:
         return
     peaks = load_peaks()
@@ -304,6 +341,7 @@ def run_ours(args, rank, world, local_rank):
                 "ms_per_step": e2e_ms},
         "clocks": clocks,
         "cpu_baseline": cpu,
+        "small_m": small_m,
     }
     print(json.dumps(line), flush=True)
 
@@ -315,6 +353,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-small-m", action="store_true")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

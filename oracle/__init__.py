@@ -35,5 +35,6 @@ from .nf4_ref import (  # noqa: F401
     quantize_nf4,
     dequantize_nf4,
     dequantize_scales,
+    dequantize_at,
 )
 from .linear_ref import lora_linear_forward, lora_linear_backward  # noqa: F401

@@ -184,6 +184,44 @@ def dequantize_nf4(codes: np.ndarray, absmax_q: np.ndarray, absmax_scale: np.nda
     return bf16_round(w32)
 
 
+def dequantize_at(w: np.ndarray, flat_idx: np.ndarray, block: int = BLOCK, group: int = GROUP) -> np.ndarray:
+    """Quantize-then-dequantize only the elements at ``flat_idx`` of ``w``.
+
+    Same definitions as :func:`quantize_nf4` followed by
+    :func:`dequantize_nf4`, evaluated only where needed: every block absmax
+    and group maximum is computed (they scale the requested elements), the
+    nearest level and the bf16 product only for the requested elements.
+    Used to check large layers on sampled outputs.
+    """
+    x = np.asarray(w, dtype=np.float32).reshape(-1)
+    n = x.size
+    nb = -(-n // block)
+    padded = np.zeros(nb * block, dtype=np.float32)
+    padded[:n] = x
+    c = np.abs(padded).reshape(nb, block).max(axis=1).astype(np.float32)
+    nb2 = -(-nb // group)
+    cpad = np.zeros(nb2 * group, dtype=np.float32)
+    cpad[:nb] = c
+    c1 = cpad.reshape(nb2, group).max(axis=1).astype(np.float32)
+
+    idx = np.asarray(flat_idx, dtype=np.int64).reshape(-1)
+    b = idx // block
+    cb = c[b]
+    with np.errstate(invalid="ignore", divide="ignore"):
+        normed = (x[idx].astype(np.float64) / cb.astype(np.float64)).astype(np.float32)
+    normed = np.where(cb == 0, np.float32(0.0), normed)
+    q = nf4_codebook()
+    code = _nearest_index(normed, q)
+    c1b = c1[b // group]
+    with np.errstate(invalid="ignore", divide="ignore"):
+        n2 = (cb.astype(np.float64) / c1b.astype(np.float64)).astype(np.float32)
+    n2 = np.where(c1b == 0, np.float32(0.0), n2)
+    code2 = _nearest_index(n2, _level2_table())
+    a = (_level2_table()[code2].astype(np.float64) * c1b.astype(np.float64)).astype(np.float32)
+    w32 = (q.astype(np.float64)[code] * a.astype(np.float64)).astype(np.float32)
+    return bf16_round(w32)
+
+
 def bits_per_parameter(numel: int, block: int = BLOCK, group: int = GROUP) -> float:
     """Stored bits per weight of the packed format (codes + both constant levels)."""
     nb = -(-numel // block)
@@ -199,6 +237,6 @@ def max_half_gap() -> float:
 
 __all__ = [
     "BLOCK", "GROUP", "ZERO_CODE", "nf4_codebook", "bf16_round", "bf16_bits",
-    "quantize_nf4", "dequantize_scales", "dequantize_nf4", "bits_per_parameter",
+    "quantize_nf4", "dequantize_scales", "dequantize_nf4", "dequantize_at", "bits_per_parameter",
     "max_half_gap",
 ]

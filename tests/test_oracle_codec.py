@@ -17,7 +17,7 @@ from fractions import Fraction
 import numpy as np
 import pytest
 
-from oracle import nf4_codebook, quantize_nf4, dequantize_nf4, dequantize_scales, bf16_round
+from oracle import nf4_codebook, quantize_nf4, dequantize_nf4, dequantize_scales, dequantize_at, bf16_round
 from oracle.nf4_ref import bits_per_parameter, max_half_gap
 from tests.exact import frac, rn_f32, rn_bf16
 
@@ -186,3 +186,14 @@ def test_bits_per_parameter_closed_form():
     x = np.zeros(n, np.float32)
     packed, code2, c1 = quantize_nf4(x[: 64 * 256 * 4])
     assert packed.size == 64 * 256 * 4 // 2 and code2.size == 256 * 4 and c1.size == 4
+
+
+def test_dequantize_at_equals_full_path():
+    rng = np.random.default_rng(21)
+    n = 64 * 256 * 5 + 100
+    x = bf16_values(rng, n, 0.03)
+    x[64 * 300:64 * 301] = 0.0
+    packed, code2, c1 = quantize_nf4(x)
+    full = dequantize_nf4(packed, code2, c1, n)
+    idx = np.concatenate([rng.choice(n, 3000, replace=False), [0, n - 1, 64 * 300 + 5]])
+    np.testing.assert_array_equal(dequantize_at(x, idx).view(np.uint32), full[idx].view(np.uint32))
