@@ -194,16 +194,27 @@ def small_m_sweep(q, synthetic, dev, flush, iters=10):
                 q.qlora_linear_fwd(X, Wp, A, B, 0.25, workspace=ws, Y=Y, T_save=T)
             stream = torch.cuda.current_stream()
             evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(iters)]
+            q.qlora_profile_start()
             for i in range(iters):
                 flush.zero_()
                 evs[i][0].record(stream)
                 q.qlora_linear_fwd(X, Wp, A, B, 0.25, workspace=ws, Y=Y, T_save=T)
                 evs[i][1].record(stream)
             torch.cuda.synchronize()
+            prof = q.qlora_profile_stop()
             us = sorted(a.elapsed_time(b) * 1e3 for a, b in evs)[iters // 2]
             gbs = nf4_bytes / (us * 1e-6) / 1e9
-            out.append({"N": N, "K": 8192, "M": M, "us": us, "nf4_weight_gbs": gbs,
-                        "frac_hbm": gbs / peaks["hbm_gbs"], "nf4_bytes": nf4_bytes})
+            ent = {"N": N, "K": 8192, "M": M, "us": us, "nf4_weight_gbs": gbs,
+                   "frac_hbm": gbs / peaks["hbm_gbs"], "nf4_bytes": nf4_bytes}
+            # The weight-streaming kernel alone (mean over the timed calls).
+            for name, (ms, calls, _) in prof.items():
+                if name in ("small_m_nf4_fwd", "fused_nf4_fwd"):
+                    k_us = ms * 1e3 / max(calls, 1)
+                    ent.update({"kernel": name, "kernel_us": k_us,
+                                "kernel_frac_hbm": nf4_bytes / (k_us * 1e-6) / 1e9 / peaks["hbm_gbs"]})
+                elif name == "lora_down_xa":
+                    ent["lora_down_us"] = ms * 1e3 / max(calls, 1)
+            out.append(ent)
     return out
 
 

@@ -34,18 +34,19 @@ constexpr size_t kStatusBytes = 256;
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // Workspace: [status word (256 B)][T pair: bf16 M x 2rp][U pair: bf16 M x 2rp]
+// and, when M <= kSmallMMax, [small-M counters and partial tiles].
 struct WsLayout {
-  size_t t_off, u_off, total;
+  size_t t_off, u_off, sm_off, total;
 };
 
 WsLayout ws_layout(int64_t M, int64_t K, int64_t N, int r) {
   (void)K;
-  (void)N;
   WsLayout w{};
   const size_t pair_bytes = round_up(static_cast<size_t>(M) * 2 * lora_pad(r) * 2, 256);
   w.t_off = kStatusBytes;
   w.u_off = w.t_off + pair_bytes;
-  w.total = w.u_off + pair_bytes;
+  w.sm_off = w.u_off + pair_bytes;
+  w.total = w.sm_off + (M <= kSmallMMax ? round_up(small_m_workspace_bytes(M, N, r), 256) : 0);
   return w;
 }
 
@@ -193,13 +194,23 @@ qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, int64_t K, int64_t N
 
   uint16_t* Tpair = reinterpret_cast<uint16_t*>(ws + wl.t_off);
 
+  if (M <= kSmallMMax) {
+    // One launch: T, its pair and Y.
+    ProfScope p0(st, "small_m_nf4_fwd", 1);
+    const cudaError_t e = launch_small_m_fwd(X, codes, absmax_q, absmax_scale, A, B, M, K, N, r, scale, Y, T_save,
+                                             Tpair, ws + wl.sm_off, status, P, st);
+    p0.done();
+    return e == cudaSuccess ? QLORA_OK : cuda_fail(e);
+  }
   ProfScope p1(st, "lora_down_xa", 1);
   cudaError_t e = launch_skinny(SkinnyKind::kXA, X, A, M, K, N, r, scale, SkinnyOut{T_save, Tpair}, status, st);
   p1.done();
   if (e != cudaSuccess) return cuda_fail(e);
-  ProfScope p2(st, "fused_nf4_fwd", 1);
-  e = launch_fused_fwd(X, codes, absmax_q, absmax_scale, Tpair, B, M, K, N, r, Y, status, P, st);
-  p2.done();
+  {
+    ProfScope p2(st, "fused_nf4_fwd", 1);
+    e = launch_fused_fwd(X, codes, absmax_q, absmax_scale, Tpair, B, M, K, N, r, Y, status, P, st);
+    p2.done();
+  }
   if (e != cudaSuccess) return cuda_fail(e);
   return QLORA_OK;
 }

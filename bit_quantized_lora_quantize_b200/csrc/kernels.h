@@ -32,6 +32,17 @@ cudaError_t launch_fused_dx(const uint16_t* dY, const uint8_t* codes, const uint
                             const float* absmax_scale, const uint16_t* Upair, const uint16_t* A, int64_t M, int64_t K,
                             int64_t N, int r, uint16_t* dX, int* status, const Nf4Params& P, cudaStream_t stream);
 
+// Small-M forward (M <= kSmallMMax tokens): the whole forward (T = s X A, its
+// pair and Y) in one launch of a persistent weight-streaming kernel.
+// `scratch` holds small_m_workspace_bytes(M, N, r) bytes, zero before the
+// first call; the kernel leaves its counters at zero when it completes.
+constexpr int64_t kSmallMMax = 128;
+size_t small_m_workspace_bytes(int64_t M, int64_t N, int r);
+cudaError_t launch_small_m_fwd(const uint16_t* X, const uint8_t* codes, const uint8_t* absmax_q,
+                               const float* absmax_scale, const uint16_t* A, const uint16_t* B, int64_t M,
+                               int64_t K, int64_t N, int r, float scale, uint16_t* Y, float* T_save, uint16_t* Tpair,
+                               void* scratch, int* status, const Nf4Params& P, cudaStream_t stream);
+
 // Rank-r products (reduction split over the CTAs of a cluster, partial tiles
 // summed in rank order through distributed shared memory):
 //   kXA   T  = s * X A          [M, r]   -> f32 (may be null) and pair

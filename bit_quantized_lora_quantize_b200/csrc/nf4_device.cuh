@@ -68,22 +68,31 @@ __device__ __forceinline__ Nf4Lut make_lut(const Nf4Params& P, float a) {
 // One 32-bit word of packed codes (byte j holds elements 2j in the high
 // nibble and 2j+1 in the low nibble) -> 8 bf16 values in element order,
 // as four bf16x2 words (lower element in the low half).
+//
+// prmt reads only the low 16 bits of its selector, one nibble per output
+// byte; a nibble with bit 3 set returns a sign-replicated byte instead of a
+// table byte.  The low table (entries 0-7) is therefore indexed with the code
+// word itself -- codes 8-15 give junk there, which the select discards -- and
+// the high table (entries 8-15) with the word XOR 0x8888...; the upper half of
+// the word is brought down with a multiply-high so that the shift runs on
+// the multiply pipe rather than the logic pipe.
 __device__ __forceinline__ void decode8(const Nf4Lut& L, uint32_t w, uint32_t (&out)[4]) {
   const uint32_t w4 = w << 4;
   // Byte k of the mask is 0xFF when the code at nibble k has bit 3 set
   // (prmt sign-replicate mode on the byte that carries that bit at its top).
   const uint32_t m0 = prmt(w, w4, 0x9D8C);
   const uint32_t m1 = prmt(w, w4, 0xBFAE);
-  const uint32_t s0 = w & 0x7777u;
-  const uint32_t s1 = (w >> 16) & 0x7777u;
+  const uint32_t wx = w ^ 0x88888888u;
+  const uint32_t wh = __umulhi(w, 0x10000u);   // w >> 16
+  const uint32_t wxh = __umulhi(wx, 0x10000u);
   // Nibbles 0..3 hold elements 1, 0, 3, 2.
-  uint32_t lo = lop3_sel(prmt(L.la0, L.la1, s0), prmt(L.lb0, L.lb1, s0), m0);
-  uint32_t hi = lop3_sel(prmt(L.ha0, L.ha1, s0), prmt(L.hb0, L.hb1, s0), m0);
+  uint32_t lo = lop3_sel(prmt(L.la0, L.la1, w), prmt(L.lb0, L.lb1, wx), m0);
+  uint32_t hi = lop3_sel(prmt(L.ha0, L.ha1, w), prmt(L.hb0, L.hb1, wx), m0);
   out[0] = prmt(lo, hi, 0x4051);
   out[1] = prmt(lo, hi, 0x6273);
   // Nibbles 4..7 hold elements 5, 4, 7, 6.
-  lo = lop3_sel(prmt(L.la0, L.la1, s1), prmt(L.lb0, L.lb1, s1), m1);
-  hi = lop3_sel(prmt(L.ha0, L.ha1, s1), prmt(L.hb0, L.hb1, s1), m1);
+  lo = lop3_sel(prmt(L.la0, L.la1, wh), prmt(L.lb0, L.lb1, wxh), m1);
+  hi = lop3_sel(prmt(L.ha0, L.ha1, wh), prmt(L.hb0, L.hb1, wxh), m1);
   out[2] = prmt(lo, hi, 0x4051);
   out[3] = prmt(lo, hi, 0x6273);
 }

@@ -123,24 +123,35 @@ def qlora_nf4_codebook() -> list:
     return list(buf)
 
 
-def qlora_quantize_nf4(W: torch.Tensor) -> PackedNF4:
-    """Quantize a bf16 CUDA tensor (any shape, flattened row-major)."""
+def qlora_quantize_nf4(W: torch.Tensor, out: PackedNF4 = None) -> PackedNF4:
+    """Quantize a bf16 CUDA tensor (any shape, flattened row-major).  `out`,
+    if given, is a PackedNF4 of the same element count whose buffers are
+    overwritten."""
     _require_cuda(W)
     if W.dtype != torch.bfloat16:
         raise ValueError("W must be bfloat16")
     n = W.numel()
     nc, nb, nb2 = packed_sizes(n)
     dev = W.device
-    codes = torch.empty(max(nc, 16), dtype=torch.uint8, device=dev)[:nc]
-    aq = torch.empty(nb, dtype=torch.uint8, device=dev)
-    sc = torch.empty(nb2, dtype=torch.float32, device=dev)
+    if out is None:
+        codes = torch.empty(max(nc, 16), dtype=torch.uint8, device=dev)[:nc]
+        aq = torch.empty(nb, dtype=torch.uint8, device=dev)
+        sc = torch.empty(nb2, dtype=torch.float32, device=dev)
+    else:
+        codes, aq, sc = out.codes, out.absmax_q, out.absmax_scale
+        if (codes.numel(), aq.numel(), sc.numel()) != (nc, nb, nb2):
+            raise ValueError("out does not hold a weight of this size")
+        _require_cuda(codes, aq, sc)
     _check("qlora_quantize_nf4", lib().qlora_quantize_nf4(_ptr(W), n, _ptr(codes), _ptr(aq), _ptr(sc), _stream()))
     return PackedNF4(codes, aq, sc, tuple(W.shape))
 
 
-def qlora_dequantize_nf4(p: PackedNF4) -> torch.Tensor:
+def qlora_dequantize_nf4(p: PackedNF4, out: torch.Tensor = None) -> torch.Tensor:
     _require_cuda(p.codes, p.absmax_q, p.absmax_scale)
-    out = torch.empty(p.shape, dtype=torch.bfloat16, device=p.codes.device)
+    if out is None:
+        out = torch.empty(p.shape, dtype=torch.bfloat16, device=p.codes.device)
+    elif out.dtype != torch.bfloat16 or out.numel() != p.numel or not out.is_contiguous():
+        raise ValueError("out must be a contiguous bf16 tensor of the weight's size")
     _check("qlora_dequantize_nf4", lib().qlora_dequantize_nf4(_ptr(p.codes), _ptr(p.absmax_q), _ptr(p.absmax_scale),
                                                               p.numel, _ptr(out), _stream()))
     return out

@@ -115,11 +115,19 @@ QLORA_API qlora_status qlora_dequantize_nf4(const uint8_t* codes, const uint8_t*
  *   Y             out  bf16[M x N]
  *   T_save        out  float[M x r]
  *   workspace     in/out device scratch of at least qlora_workspace_bytes(M,K,N,r)
- *                 bytes; contents on entry are ignored, except that the
- *                 first 256 bytes hold the status word read by
- *                 qlora_check_status (clear them once with zeros).
+ *                 bytes, filled with zeros once before its first use.  It
+ *                 holds the status word read by qlora_check_status (first
+ *                 256 bytes) and counters that every call leaves at zero;
+ *                 everything else is overwritten before it is read.  After
+ *                 qlora_check_status reports QLORA_ERR_TIMEOUT, fill it with
+ *                 zeros again before the next call.
  * Supported: K % 64 == 0, N % 8 == 0, r % 8 == 0 with 8 <= r <= 128,
  * M, N, K < 2^31.  Otherwise QLORA_ERR_UNSUPPORTED.
+ * For M <= 128 the whole forward is one kernel whose thread blocks wait for
+ * one another (cooperative launch: all of them must be resident at once);
+ * if the device cannot hold them next to other work the call returns
+ * QLORA_ERR_CUDA and launches nothing.  Sums are taken in a fixed order:
+ * results are bit-reproducible run to run.
  */
 QLORA_API qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, int64_t K, int64_t N, const uint8_t* codes,
                               const uint8_t* absmax_q, const float* absmax_scale, const uint16_t* A,
@@ -154,8 +162,10 @@ QLORA_API qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, c
  * callback, on a path where the framework forbids allocation, or in an
  * embedding that owns all device memory up front).  The QLoRA pages have no
  * counterpart to this call; it exists for those callers only.
- *   Same arguments, outputs, supported shapes and results as
- *   qlora_linear_fwd, minus workspace/ws_bytes.  The call allocates nothing:
+ *   Same arguments, outputs and supported shapes as qlora_linear_fwd, minus
+ *   workspace/ws_bytes; the results agree with qlora_linear_fwd to within
+ *   float32 summation order (for M <= 128 the two use different kernels).
+ *   The call allocates nothing:
  *   its scratch is one fixed 16 MiB device array inside this library, which
  *   every GPU that loads the library keeps until the process exits.
  *   - Shapes whose forward scratch (status word + bf16 pair of T, i.e.

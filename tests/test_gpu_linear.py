@@ -54,6 +54,33 @@ def test_ragged_shapes(M, K, N, r):
     check_full(case, run_gpu(case))
 
 
+# Forward shapes of the weight-streaming path (M <= 128 tokens): every token
+# padding width (16, 32, 64, 128), ragged weight tiles (N % 128 != 0), one
+# reduction block (K = 64), LoRA ranks with one or two 64-column blocks, and
+# products whose 128-row tiles are split over several CTAs.
+@pytest.mark.parametrize("M,K,N,r", [(2, 64, 136, 8), (17, 4096, 1024, 64), (33, 1536, 1000, 72),
+                                     (64, 2048, 2056, 128), (65, 640, 392, 16), (128, 4096, 776, 64),
+                                     (8, 11008, 512, 64)])
+def test_small_m_shapes(M, K, N, r):
+    case = synthetic.linear_case(M, K, N, r, 0.5, seed=3 * M + K + N + r)
+    check_full(case, run_gpu(case))
+
+
+def test_small_m_repeated_calls_are_identical():
+    """Split tiles are summed through per-tile counters that each call resets:
+    three calls on one workspace give the same bits."""
+    case = synthetic.linear_case(16, 4096, 2048, 64, 0.25, seed=19)
+    Wp = q.qlora_quantize_nf4(case.W.to(DEV))
+    X, A, B = (t.to(DEV) for t in (case.X, case.A, case.B))
+    ws = q.new_workspace(case.M, case.K, case.N, case.r, DEV)
+    outs = [q.qlora_linear_fwd(X, Wp, A, B, case.scale, workspace=ws)[0] for _ in range(3)]
+    assert q.qlora_check_status(ws) == 0
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
+    Wdq = oracle_wdq(case)
+    Y, _ = lora_linear_forward(f64(case.X), Wdq, f64(case.A), f64(case.B), case.scale)
+    assert_close_rms(f64(outs[0]), Y, "Y")
+
+
 def test_special_cases_exact():
     base = synthetic.linear_case(192, 256, 320, 16, 1.0, seed=21)
     # B = 0: no gradient reaches A, bit-exactly; Y is the frozen product.
