@@ -17,8 +17,9 @@
 //
 // Per CTA: warp 0 issues TMA (activation rows and LoRA tiles signal the
 // leader CTA's barrier, packed codes a local one; no multicast loads), warp 1
-// allocates TMEM (both CTAs) and, in the leader only, issues the MMAs and
-// commits them to both CTAs' barriers; warps 4-7 decode the even stages and
+// allocates TMEM (both CTAs); in the leader only, warps 1 and 2 issue the MMAs
+// of the two accumulators and commit them to both CTAs' barriers; warps 4-7
+// decode the even stages and
 // warps 8-11 the odd ones (one 64-weight block per thread per stage), then
 // all eight drain the two 128 x 256 fp32 accumulators.
 #include <algorithm>
@@ -165,10 +166,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&cfull[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&empty[s], 2);  // one commit from each MMA issuer
       mbar_init(&decoded[s], 2 * kDecWarps);
     }
-    mbar_init(acc_full, 1);
+    mbar_init(acc_full, 2);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -247,13 +248,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == 1 || warp == 2) {
     // ------------------------------------------------------------ MMA (leader)
+    // One tcgen05.mma takes its issuing thread about as long as the tensor
+    // cores take to execute it at this tile size, so the two M = 256
+    // accumulators are fed by two threads: warp 1 issues the first, warp 2 the
+    // second; each commits to the stage and accumulator barriers (count 2).
     if (lane == 0 && rank == 0) {
+      const int h = warp - 1;
       const WaitCtx ctx{abort_flag, args.status, 22};
       // M = 256 across the pair, N = 256 (each CTA supplies 128 columns of B).
       const uint32_t idesc_main = idesc_bf16_f32(256, 256, false, MNB);
       const uint32_t idesc_lora = idesc_bf16_f32(256, 256, false, !MNB);
+      const uint32_t d = tmem_acc + h * 256;
       bool ok = true;
       for (int i = 0; i < total && ok; ++i) {
         const int s = i % kStages;
@@ -262,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(&full[s], ph, ctx)) { ok = false; break; }
         if (main_stage && !mbar_wait(&decoded[s], ph, ctx)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t a_base = smem_u32(sA + s * L::kA);
+        const uint32_t a_base = smem_u32(sA + s * L::kA) + h * 16384;
         const uint32_t b_base = smem_u32(sB + s * L::kB);
         const bool b_mn = main_stage ? MNB : !MNB;
 #pragma unroll
@@ -271,8 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                       : smem_desc_sw128(b_base + kk * 32, 16, 1024);
           const uint32_t idesc = main_stage ? idesc_main : idesc_lora;
           const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
-          umma_pair(tmem_acc, smem_desc_sw128(a_base + kk * 32, 16, 1024), bdesc, idesc, acc);
-          umma_pair(tmem_acc + 256, smem_desc_sw128(a_base + 16384 + kk * 32, 16, 1024), bdesc, idesc, acc);
+          umma_pair(d, smem_desc_sw128(a_base + kk * 32, 16, 1024), bdesc, idesc, acc);
         }
         umma_commit_pair(&empty[s]);
       }

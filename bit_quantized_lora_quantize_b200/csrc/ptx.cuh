@@ -47,6 +47,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// As mbar_try_wait, but the thread may stay suspended in hardware for up to
+// `hint_ns` (it resumes as soon as the phase completes): a waiting warp then
+// takes no issue slots from the warps that are working.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Every wait in the kernels is bounded.  A wait that gives up sets the CTA's
 // abort flag (shared memory) and the device status word, and returns false;
 // all other waits of the CTA then fall through, so that every thread still
@@ -65,7 +80,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
   while (true) {
 #pragma unroll 1
     for (int i = 0; i < 32; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
+      if (mbar_try_wait_sleep(bar, parity, 20000)) return true;
     if (*ctx.abort_flag) return false;
     if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
       *ctx.abort_flag = 1;

@@ -42,7 +42,7 @@
 // not depend on timing.  Counters are returned to zero by the CTA that
 // finishes with them.
 //
-// Warp roles: 0 TMA producer, 1 TMEM allocation and MMA issue, 2, 3 and 24
+// Warp roles: 0 and 25-27 TMA producers, 1 TMEM allocation and MMA issue, 2, 3 and 24
 // further MMA issuers (with few tokens an MMA is too small to cover its own
 // issue time, so up to four threads issue them), 4-7 epilogue (T partials
 // and tree, tile partials), 8-23 decoders (four groups of four warps taking
@@ -69,7 +69,12 @@ constexpr int kTileRows = 128;      // weight rows per tile (MMA M)
 constexpr int kGroups = 4;          // decoder groups (weight units round robin)
 constexpr int kDecWarp0 = 8;        // decoder warps 8 .. 8 + 4 kGroups - 1
 constexpr int kIssuerWarp3 = kDecWarp0 + 4 * kGroups;  // the fourth MMA issuer
-constexpr int kThreads = (kIssuerWarp3 + 1) * 32;
+// One TMA issue takes its thread ~140 cycles, about as long as a weight unit
+// takes to stream at the HBM rate, so the weight units' copies are issued by
+// four producer threads (warp 0 and these three warps), round robin.
+constexpr int kProducers = 4;
+constexpr int kProducerWarp1 = kIssuerWarp3 + 1;
+constexpr int kThreads = (kProducerWarp1 + kProducers - 1) * 32;
 constexpr int kLoraSlots = 2;       // ring for T and LoRA units
 constexpr int kPrefetch = 4;        // block constants are loaded this many own units ahead
 constexpr int kMaxGrid = 256;       // workspace is sized for this many CTAs
@@ -88,7 +93,9 @@ struct SmallLayout {
   static constexpr int kPairTab = 256 * 16 * 8;        // 32 KB: code byte -> two float32 levels, 16 copies
   static constexpr int kFixed = kLoraSlots * kLSlot + kPairTab + 1024 /*lvl2*/ + 1024 /*barriers*/;
   static constexpr int kStagesRaw = (kSmemBudget - kFixed) / kSlot;
-  static constexpr int kStages = std::min(24, kStagesRaw / kGroups * kGroups);  // each decoder group owns fixed slots
+  // Multiple of the decoder-group and producer counts: each ring slot always
+  // belongs to the same decoder group and the same producer.
+  static constexpr int kStages = std::min(24, kStagesRaw / kGroups * kGroups);
   static constexpr int offSlots = 0;
   static constexpr int offLora = offSlots + kStages * kSlot;
   static constexpr int offPairTab = offLora + kLoraSlots * kLSlot;
@@ -119,6 +126,7 @@ struct SmallLayout {
   static constexpr bool kDefer = false;
   static_assert(kStages >= kGroups && kASlots >= kGroups, "one unit in flight per decoder group");
   static_assert(kStages % kGroups == 0 && kASlots % kGroups == 0, "decoder groups own fixed slots");
+  static_assert(kStages % kProducers == 0, "producers own fixed slots");
   static_assert(kASlots % kIssuers == 0, "an A slot is always consumed by the same issuer");
   static_assert(kAccCols + kASlots * 32 <= 512, "tensor memory budget");
 };
@@ -303,8 +311,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
+  if (warp == 0 || warp >= kProducerWarp1) {
+    // ------------------------------------------------------------ producers
+    // Producer p issues the copies of weight units jm = p (mod kProducers);
+    // producer 0 also issues every T and LoRA unit.
+    const int p = warp == 0 ? 0 : warp - kProducerWarp1 + 1;
     if (lane == 0) {
       const WaitCtx ctx{abort_flag, args.status, 41};
       int jm = 0, jl = 0;
@@ -317,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++jl;
         return &lfull[ls];
       };
-      for (int64_t k = tk0; k < tk1 && ok; ++k) {
+      for (int64_t k = tk0; k < tk1 && ok && p == 0; ++k) {
         uint8_t* dst;
         uint64_t* bar = lora_slot(dst);
         if (!bar) { ok = false; break; }
@@ -327,26 +338,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_2d(&tmX, bar, dst + L::kAt, y, 0);
       }
       int t = static_cast<int>(mx0 / KB), kb = static_cast<int>(mx0 % KB);
-      for (int64_t x = mx0; x < mx1 && ok; ++x) {
-        const int s = jm % S;
-        if (!mbar_wait(&consumed[s], ((jm / S) & 1) ^ 1, ctx)) { ok = false; break; }
-        uint8_t* dst = sSlots + s * L::kSlot;
-        mbar_arrive_expect_tx(&full[s], L::kSlot);
-        tma_load_2d(&tmC, &full[s], dst, kb * 32, t * kTileRows);
-        tma_load_2d(&tmX, &full[s], dst + L::kCodes, kb * kDepth, 0);
-        ++jm;
+      for (int64_t x = mx0; x < mx1 && ok; ++x, ++jm) {
+        if (jm % kProducers == p) {
+          const int s = jm % S;
+          if (!mbar_wait(&consumed[s], ((jm / S) & 1) ^ 1, ctx)) { ok = false; break; }
+          uint8_t* dst = sSlots + s * L::kSlot;
+          mbar_arrive_expect_tx(&full[s], L::kSlot);
+          tma_load_2d(&tmC, &full[s], dst, kb * 32, t * kTileRows);
+          tma_load_2d(&tmX, &full[s], dst + L::kCodes, kb * kDepth, 0);
+        }
         if (++kb == KB) {
           kb = 0;
           ++t;
         }
       }
-      if (ok && lt0 < lt1) {
+      if (ok && lt0 < lt1 && p == 0) {
         // The T pair is written by another CTA with ordinary stores and read
         // here by TMA: acquire the ready count, then order the async proxy.
         ok = wait_t_ready(args, ctx);
         fence_proxy_async_global();
       }
-      for (int tt = lt0; tt < lt1 && ok; ++tt) {
+      for (int tt = lt0; tt < lt1 && ok && p == 0; ++tt) {
         for (int lk = 0; lk < args.L; ++lk) {
           uint8_t* dst;
           uint64_t* bar = lora_slot(dst);
@@ -358,11 +370,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (*abort_flag) {
-        // Let the copies already issued land before the CTA exits.
+        // Let the copies this thread issued land before the CTA exits.
         const uint64_t t0 = globaltimer_ns();
         for (int i = (jm > S ? jm - S : 0); i < jm; ++i)
-          while (!mbar_try_wait(&full[i % S], (i / S) & 1) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
-          }
+          if (i % kProducers == p)
+            while (!mbar_try_wait(&full[i % S], (i / S) & 1) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
+            }
         for (int i = (jl > kLoraSlots ? jl - kLoraSlots : 0); i < jl; ++i)
           while (!mbar_try_wait(&lfull[i % kLoraSlots], (i / kLoraSlots) & 1) &&
                  globaltimer_ns() - t0 < kWaitTimeoutNs) {
