@@ -264,17 +264,25 @@ def run_ours(args, rank, world, local_rank):
         dist.barrier()
     torch.cuda.synchronize()
     sampler.start()
-    q.qlora_profile_start()
     for i in range(args.steps):
         flush.zero_()
         evs[i][0].record(stream)
         step()
         evs[i][1].record(stream)
     torch.cuda.synchronize()
-    prof = q.qlora_profile_stop()
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
+    # Per-kernel durations (roofline, kernel table): the same K steps again
+    # with CUDA events recorded around every launch on the launching stream.
+    # Kept out of the timed steps above, because an event between two kernels
+    # stops the next one from starting before the previous one ends.
+    q.qlora_profile_start()
+    for i in range(args.steps):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    prof = q.qlora_profile_stop()
     step_ms = [a.elapsed_time(b) for a, b in evs]
     total_ms = sum(step_ms)
     t = torch.tensor([total_ms], dtype=torch.float64, device=dev)

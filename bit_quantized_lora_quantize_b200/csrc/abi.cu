@@ -238,15 +238,12 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   const Nf4Params& P = nf4_params();
 
+  // Launch order puts each kernel right after the one whose output it needs
+  // (the kernels start early and wait for their predecessor only there):
+  // U -> dX (U pair in its last stages) -> dA (U pair) -> T pair -> dB.
   ProfScope p1(st, "lora_u_dybt", 1);
   cudaError_t e = launch_skinny(SkinnyKind::kDyBt, dY, B, M, K, N, r, scale, SkinnyOut{nullptr, Upair}, status, st);
   p1.done();
-  if (e != cudaSuccess) return cuda_fail(e);
-  ProfScope p2(st, "lora_db_ttdy", 2);
-  e = launch_split_pair(T_save, M, r, Tpair, st);
-  if (e == cudaSuccess)
-    e = launch_skinny(SkinnyKind::kTtDy, dY, Tpair, M, K, N, r, 1.0f, SkinnyOut{dB, nullptr}, status, st);
-  p2.done();
   if (e != cudaSuccess) return cuda_fail(e);
   ProfScope p3(st, "fused_nf4_dx", 1);
   e = launch_fused_dx(dY, codes, absmax_q, absmax_scale, Upair, A, M, K, N, r, dX, status, P, st);
@@ -255,6 +252,12 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float
   ProfScope p4(st, "lora_da_xtu", 1);
   e = launch_skinny(SkinnyKind::kXtU, X, Upair, M, K, N, r, 1.0f, SkinnyOut{dA, nullptr}, status, st);
   p4.done();
+  if (e != cudaSuccess) return cuda_fail(e);
+  ProfScope p2(st, "lora_db_ttdy", 2);
+  e = launch_split_pair(T_save, M, r, Tpair, st);
+  if (e == cudaSuccess)
+    e = launch_skinny(SkinnyKind::kTtDy, dY, Tpair, M, K, N, r, 1.0f, SkinnyOut{dB, nullptr}, status, st);
+  p2.done();
   if (e != cudaSuccess) return cuda_fail(e);
   return QLORA_OK;
 }

@@ -188,6 +188,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   cluster_sync_all();  // the leader's barriers exist before the peer signals them
   tc_fence_after();
   const uint32_t tmem_acc = *tmem_slot;
+  // The previous kernel in the stream produces only the LoRA intermediate
+  // (T or U pair), read in the last stages: everything else may start now.
+  griddep_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -222,6 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           const int lk = i - args.nkb;
           const int lb = (lk * kDepth) % args.lora_mod;
+          if (lk == 0) griddep_wait();  // the pair is the previous kernel's output
           if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * (L::kA + L::kB));
           tma_load_2d_pair(&tmA2, full_leader, a_dst, lk * kDepth, row0);
           tma_load_2d_pair(&tmA2, full_leader, a_dst + 16384, lk * kDepth, row0 + 256);
@@ -462,13 +466,14 @@ cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& c, const CUtens
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = L::kDynamic;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1] = pdl_attribute();
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, kern, a, c, a2, b2, abs, args);
 }
 

@@ -9,6 +9,17 @@
 
 namespace qlora {
 
+// Launch attribute that lets a kernel start before its predecessor in the
+// stream has ended (programmatic dependent launch).  Every kernel launched
+// with it calls griddep_wait before it reads anything its predecessor writes
+// and before it writes anything its predecessor reads.
+inline cudaLaunchAttribute pdl_attribute() {
+  cudaLaunchAttribute a{};
+  a.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  a.val.programmaticStreamSerializationAllowed = 1;
+  return a;
+}
+
 cudaError_t launch_quantize_nf4(const uint16_t* W, int64_t numel, uint8_t* codes, uint8_t* absmax_q,
                                 float* absmax_scale, const Nf4Params& P, cudaStream_t stream);
 

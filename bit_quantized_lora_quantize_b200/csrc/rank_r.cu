@@ -167,6 +167,10 @@ __global__ void __launch_bounds__(kRankThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_acc = *tmem_slot;
+  // The set-up above overlaps the previous kernel; the operands may be its
+  // outputs, so every thread waits for it here.
+  griddep_wait();
+  griddep_launch_dependents();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -266,20 +270,34 @@ __global__ void __launch_bounds__(kRankThreads, 1)
   const int c4 = a.rp / 4;  // output column groups
   const uint32_t p_local = smem_u32(P);
   const bool rows_fastest = a.kind == static_cast<int>(SkinnyKind::kTtDy);
+  // All peers' loads of an item are issued before any is used, so the
+  // distributed-shared-memory round trips overlap; the sums then run in rank
+  // order (fixed, hence bit-reproducible).
+  uint32_t peer[kMaxSplits];
+#pragma unroll
+  for (int k = 0; k < kMaxSplits; ++k) peer[k] = k < S ? peer_addr(p_local, k) : p_local;
   for (int t = threadIdx.x; t < R * c4; t += kRankThreads) {
     const int rr = rows_fastest ? (t % R) : (t / c4);
     const int jj = rows_fastest ? (t / R) : (t % c4);
     const int lrow = r0 + rr;
     const int64_t row = static_cast<int64_t>(tile) * kTile + lrow;
     const uint32_t off = static_cast<uint32_t>((lrow * L::kPStride + 4 * jj) * 4);
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f), lo = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int k = 0; k < S; ++k) {
-      const uint32_t base = peer_addr(p_local, k);
-      const float4 v = ld_peer4(base + off);
-      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-      if (consumer) {
-        const float4 w = ld_peer4(base + off + a.rp * 4);
-        lo.x += w.x; lo.y += w.y; lo.z += w.z; lo.w += w.w;
+    float4 v[kMaxSplits], w[kMaxSplits];
+#pragma unroll
+    for (int k = 0; k < kMaxSplits; ++k) {
+      if (k < S) {
+        v[k] = ld_peer4(peer[k] + off);
+        if (consumer) w[k] = ld_peer4(peer[k] + off + a.rp * 4);
+      }
+    }
+    float4 acc = v[0], lo = consumer ? w[0] : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int k = 1; k < kMaxSplits; ++k) {
+      if (k < S) {
+        acc.x += v[k].x; acc.y += v[k].y; acc.z += v[k].z; acc.w += v[k].w;
+        if (consumer) {
+          lo.x += w[k].x; lo.y += w[k].y; lo.z += w[k].z; lo.w += w[k].w;
+        }
       }
     }
     if (consumer) {
@@ -328,13 +346,14 @@ cudaError_t launch_rank_bn(const CUtensorMap& ma, const CUtensorMap& mb, const R
   cfg.blockDim = dim3(kRankThreads, 1, 1);
   cfg.dynamicSmemBytes = L::kDynamic;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = static_cast<unsigned>(a.splits);
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1] = pdl_attribute();
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, kern, ma, mb, a);
 }
 
@@ -419,6 +438,8 @@ cudaError_t launch_skinny(SkinnyKind kind, const uint16_t* P0, const uint16_t* P
 
 // bf16 pair of a float32 [rows x r] matrix.
 __global__ void split_pair_kernel(const float* __restrict__ v, int64_t rows, int r, int rp, uint16_t* __restrict__ pair) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (idx >= rows * rp) return;
   const int64_t row = idx / rp;
@@ -438,8 +459,14 @@ __global__ void split_pair_kernel(const float* __restrict__ v, int64_t rows, int
 cudaError_t launch_split_pair(const float* v, int64_t rows, int r, uint16_t* pair, cudaStream_t stream) {
   const int rp = lora_pad(r);
   const int64_t n = rows * rp;
-  split_pair_kernel<<<static_cast<unsigned>(ceil_div64(n, 256)), 256, 0, stream>>>(v, rows, r, rp, pair);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(ceil_div64(n, 256)), 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1] = {pdl_attribute()};
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, split_pair_kernel, v, rows, r, rp, pair);
 }
 
 }  // namespace qlora
