@@ -1,5 +1,6 @@
 // C ABI of the library: argument validation, workspace layout and the
 // sequence of kernel launches for each call (declared in include/qlora.h).
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -34,18 +35,22 @@ constexpr size_t kStatusBytes = 256;
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // Workspace: [status word (256 B)][T pair: bf16 M x 2rp][U pair: bf16 M x 2rp]
-// and, when M <= kSmallMMax, [small-M counters and partial tiles].
+// [partial tiles of the rank-r products (one at a time)] and, when
+// M <= kSmallMMax, [small-M counters and partial tiles].
 struct WsLayout {
-  size_t t_off, u_off, sm_off, total;
+  size_t t_off, u_off, rk_off, sm_off, total;
 };
 
 WsLayout ws_layout(int64_t M, int64_t K, int64_t N, int r) {
-  (void)K;
   WsLayout w{};
   const size_t pair_bytes = round_up(static_cast<size_t>(M) * 2 * lora_pad(r) * 2, 256);
+  size_t rank_bytes = 0;
+  for (SkinnyKind k : {SkinnyKind::kXA, SkinnyKind::kDyBt, SkinnyKind::kTtDy, SkinnyKind::kXtU})
+    rank_bytes = std::max(rank_bytes, skinny_scratch_bytes(k, M, K, N, r));
   w.t_off = kStatusBytes;
   w.u_off = w.t_off + pair_bytes;
-  w.sm_off = w.u_off + pair_bytes;
+  w.rk_off = w.u_off + pair_bytes;
+  w.sm_off = w.rk_off + round_up(rank_bytes, 256);
   w.total = w.sm_off + (M <= kSmallMMax ? round_up(small_m_workspace_bytes(M, N, r), 256) : 0);
   return w;
 }
@@ -203,7 +208,8 @@ qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, int64_t K, int64_t N
     return e == cudaSuccess ? QLORA_OK : cuda_fail(e);
   }
   ProfScope p1(st, "lora_down_xa", 1);
-  cudaError_t e = launch_skinny(SkinnyKind::kXA, X, A, M, K, N, r, scale, SkinnyOut{T_save, Tpair}, status, st);
+  float* rk = reinterpret_cast<float*>(ws + wl.rk_off);
+  cudaError_t e = launch_skinny(SkinnyKind::kXA, X, A, M, K, N, r, scale, SkinnyOut{T_save, Tpair}, rk, status, st);
   p1.done();
   if (e != cudaSuccess) return cuda_fail(e);
   {
@@ -242,7 +248,8 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float
   // (the kernels start early and wait for their predecessor only there):
   // U -> dX (U pair in its last stages) -> dA (U pair) -> T pair -> dB.
   ProfScope p1(st, "lora_u_dybt", 1);
-  cudaError_t e = launch_skinny(SkinnyKind::kDyBt, dY, B, M, K, N, r, scale, SkinnyOut{nullptr, Upair}, status, st);
+  float* rk = reinterpret_cast<float*>(ws + wl.rk_off);
+  cudaError_t e = launch_skinny(SkinnyKind::kDyBt, dY, B, M, K, N, r, scale, SkinnyOut{nullptr, Upair}, rk, status, st);
   p1.done();
   if (e != cudaSuccess) return cuda_fail(e);
   ProfScope p3(st, "fused_nf4_dx", 1);
@@ -250,13 +257,13 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float
   p3.done();
   if (e != cudaSuccess) return cuda_fail(e);
   ProfScope p4(st, "lora_da_xtu", 1);
-  e = launch_skinny(SkinnyKind::kXtU, X, Upair, M, K, N, r, 1.0f, SkinnyOut{dA, nullptr}, status, st);
+  e = launch_skinny(SkinnyKind::kXtU, X, Upair, M, K, N, r, 1.0f, SkinnyOut{dA, nullptr}, rk, status, st);
   p4.done();
   if (e != cudaSuccess) return cuda_fail(e);
   ProfScope p2(st, "lora_db_ttdy", 2);
   e = launch_split_pair(T_save, M, r, Tpair, st);
   if (e == cudaSuccess)
-    e = launch_skinny(SkinnyKind::kTtDy, dY, Tpair, M, K, N, r, 1.0f, SkinnyOut{dB, nullptr}, status, st);
+    e = launch_skinny(SkinnyKind::kTtDy, dY, Tpair, M, K, N, r, 1.0f, SkinnyOut{dB, nullptr}, rk, status, st);
   p2.done();
   if (e != cudaSuccess) return cuda_fail(e);
   return QLORA_OK;

@@ -77,8 +77,12 @@ struct SkinnyOut {
 
 SkinnyPlan plan_skinny(SkinnyKind kind, int64_t M, int64_t K, int64_t N, int r);
 
+// `scratch` (16-byte aligned, skinny_scratch_bytes of this product) holds the
+// splits' partial tiles in global memory; null keeps them in shared memory and
+// sums them through distributed shared memory instead.
+size_t skinny_scratch_bytes(SkinnyKind kind, int64_t M, int64_t K, int64_t N, int r);
 cudaError_t launch_skinny(SkinnyKind kind, const uint16_t* P0, const uint16_t* P1, int64_t M, int64_t K, int64_t N,
-                          int r, float scale, SkinnyOut out, int* status, cudaStream_t stream);
+                          int r, float scale, SkinnyOut out, float* scratch, int* status, cudaStream_t stream);
 
 // Pair matrix of a float32 [rows x r] matrix.
 cudaError_t launch_split_pair(const float* v, int64_t rows, int r, uint16_t* pair, cudaStream_t stream);

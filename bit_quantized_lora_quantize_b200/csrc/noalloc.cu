@@ -95,7 +95,7 @@ extern "C" qlora_status qlora_linear_fwd_noalloc(const uint16_t* X, int64_t M, i
   // Clear the status word: a call that timed out earlier may have left it set.
   e = cudaMemsetAsync(ws, 0, sizeof(int), st);
   if (e == cudaSuccess)
-    e = launch_skinny(SkinnyKind::kXA, X, A, M, K, N, r, scale, SkinnyOut{T_save, Tpair}, status, st);
+    e = launch_skinny(SkinnyKind::kXA, X, A, M, K, N, r, scale, SkinnyOut{T_save, Tpair}, nullptr, status, st);
   if (e == cudaSuccess)
     e = launch_fused_fwd(X, codes, absmax_q, absmax_scale, Tpair, B, M, K, N, r, Y, status, nf4_params(), st);
   return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;

@@ -51,6 +51,10 @@ struct RankArgs {
   int kind;          // SkinnyKind
   float* f32;        // T (may be null), dA, dB
   uint16_t* pair;    // T / U pair
+  // Partial tiles of the splits, [tile][split][BN / 4][128 rows] float4, or
+  // null: then each CTA keeps its partial in shared memory and the cluster
+  // reads it through distributed shared memory (slower, needs no scratch).
+  float4* scratch;
   int* status;
 };
 
@@ -241,8 +245,16 @@ __global__ void __launch_bounds__(kRankThreads, 1)
     const bool ok = (n == 0) || __all_sync(0xFFFFFFFFu, mbar_wait(acc_full, 0, ctx));
     tc_fence_after();
     float* prow = P + lrow * L::kPStride;
+    // Column group g of this row: global scratch (coalesced over rows) or
+    // the padded shared-memory row.
+    float4* grow = a.scratch ? a.scratch + (static_cast<int64_t>(tile) * a.splits + split) * (BN / 4) * kTile + lrow
+                             : nullptr;
+    auto put = [&](int g, float4 v) {
+      if (grow) grow[g * kTile] = v;
+      else *reinterpret_cast<float4*>(prow + 4 * g) = v;
+    };
     if (n == 0 || !ok) {
-      for (int j = 0; j < BN; j += 4) *reinterpret_cast<float4*>(prow + j) = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int g = 0; g < BN / 4; ++g) put(g, make_float4(0.f, 0.f, 0.f, 0.f));
     } else {
       const uint32_t t_row = tmem_acc + (static_cast<uint32_t>(q * 32) << 16);
 #pragma unroll 1
@@ -252,16 +264,16 @@ __global__ void __launch_bounds__(kRankThreads, 1)
         tmem_wait_ld();
 #pragma unroll
         for (int g = 0; g < 8; ++g)
-          *reinterpret_cast<float4*>(prow + j0 + 4 * g) =
-              make_float4(__uint_as_float(u[4 * g]), __uint_as_float(u[4 * g + 1]), __uint_as_float(u[4 * g + 2]),
-                          __uint_as_float(u[4 * g + 3]));
+          put(j0 / 4 + g, make_float4(__uint_as_float(u[4 * g]), __uint_as_float(u[4 * g + 1]),
+                                      __uint_as_float(u[4 * g + 2]), __uint_as_float(u[4 * g + 3])));
       }
     }
+    if (grow) __threadfence();
   }
 
   tc_fence_before();
   __syncthreads();
-  cluster_sync_all();  // every CTA's partial tile is in its shared memory
+  cluster_sync_all();  // every CTA's partial tile is in place (release/acquire at cluster scope)
 
   // Sum rows [r0, r1) of the S partial tiles in rank order.
   const int S = a.splits;
@@ -283,11 +295,23 @@ __global__ void __launch_bounds__(kRankThreads, 1)
     const int64_t row = static_cast<int64_t>(tile) * kTile + lrow;
     const uint32_t off = static_cast<uint32_t>((lrow * L::kPStride + 4 * jj) * 4);
     float4 v[kMaxSplits], w[kMaxSplits];
+    if (a.scratch) {
+      // Partials in global memory (L2): all loads first, then the sums.
+      const float4* base = a.scratch + static_cast<int64_t>(tile) * S * (BN / 4) * kTile + lrow;
 #pragma unroll
-    for (int k = 0; k < kMaxSplits; ++k) {
-      if (k < S) {
-        v[k] = ld_peer4(peer[k] + off);
-        if (consumer) w[k] = ld_peer4(peer[k] + off + a.rp * 4);
+      for (int k = 0; k < kMaxSplits; ++k) {
+        if (k < S) {
+          v[k] = __ldcg(base + (static_cast<int64_t>(k) * (BN / 4) + jj) * kTile);
+          if (consumer) w[k] = __ldcg(base + (static_cast<int64_t>(k) * (BN / 4) + c4 + jj) * kTile);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int k = 0; k < kMaxSplits; ++k) {
+        if (k < S) {
+          v[k] = ld_peer4(peer[k] + off);
+          if (consumer) w[k] = ld_peer4(peer[k] + off + a.rp * 4);
+        }
       }
     }
     float4 acc = v[0], lo = consumer ? w[0] : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -386,8 +410,13 @@ SkinnyPlan plan_skinny(SkinnyKind kind, int64_t M, int64_t K, int64_t N, int r) 
   return p;
 }
 
+size_t skinny_scratch_bytes(SkinnyKind kind, int64_t M, int64_t K, int64_t N, int r) {
+  const SkinnyPlan p = plan_skinny(kind, M, K, N, r);
+  return static_cast<size_t>(p.tiles) * p.splits * kTile * p.bn * 4;
+}
+
 cudaError_t launch_skinny(SkinnyKind kind, const uint16_t* P0, const uint16_t* P1, int64_t M, int64_t K, int64_t N,
-                          int r, float scale, SkinnyOut out, int* status, cudaStream_t stream) {
+                          int r, float scale, SkinnyOut out, float* scratch, int* status, cudaStream_t stream) {
   const SkinnyPlan p = plan_skinny(kind, M, K, N, r);
   const Geometry geo = geometry(kind, M, K, N);
   const int rp = lora_pad(r);
@@ -428,6 +457,7 @@ cudaError_t launch_skinny(SkinnyKind kind, const uint16_t* P0, const uint16_t* P
   a.kind = static_cast<int>(kind);
   a.f32 = out.f32;
   a.pair = out.pair;
+  a.scratch = reinterpret_cast<float4*>(scratch);
   a.status = status;
   switch (kind) {
     case SkinnyKind::kXA: return dispatch_rank<false, true>(p.bn, ma, mb, a, p.tiles, stream);
