@@ -213,9 +213,11 @@ def traffic_for(kernel: str):
         with open(path) as f:
             t = json.load(f)
         ent = t[kernel]
-        src = os.path.join(ROOT, "bit_quantized_lora_quantize_b200", "csrc", ent["source"])
-        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-        if h != ent["source_sha256_16"]:
+        hsh = hashlib.sha256()
+        for name in ent["sources"]:  # the kernel's .cu file and the headers it includes
+            with open(os.path.join(ROOT, "bit_quantized_lora_quantize_b200", "csrc", name), "rb") as f:
+                hsh.update(f.read())
+        if hsh.hexdigest()[:16] != ent["sources_sha256_16"]:
             return None
         return ent["dram_bytes_per_launch"]
     except Exception:
