@@ -24,7 +24,6 @@ import os
 import subprocess
 import sys
 import tempfile
-import threading
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -65,46 +64,48 @@ class ClockSampler:
         self.gpu = gpu_index
         self.proc = None
         self.path = None
-        self.thread = None
-        self.rows = []
-        self.stop_flag = False
+        self.poller = None
 
-    # Preferred: NVML read in a thread every ~1 ms, so that even a timed region
-    # of a few milliseconds is sampled.  Read-only queries; nothing is set.
-    def _nvml_handle(self):
-        import pynvml
+    # Preferred: NVML read every ~1 ms by a child process (a thread of this
+    # process would share the GIL with the launch loop and could go unsampled
+    # for a whole short timed region).  Read-only queries; nothing is set.
+    POLL = (
+        "import json, select, sys\n"
+        "import pynvml\n"
+        "pynvml.nvmlInit()\n"
+        "try:\n"
+        "    h = pynvml.nvmlDeviceGetHandleByPciBusId(sys.argv[1])\n"
+        "except Exception:\n"
+        "    h = pynvml.nvmlDeviceGetHandleByIndex(int(sys.argv[2]))\n"
+        "gr = getattr(pynvml, 'nvmlDeviceGetCurrentClocksEventReasons', None) or "
+        "getattr(pynvml, 'nvmlDeviceGetCurrentClocksThrottleReasons')\n"
+        "mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)\n"
+        "rows = []\n"
+        "def sample():\n"
+        "    rows.append((pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM), gr(h)))\n"
+        "sample()\n"
+        "print('ready', flush=True)\n"
+        "while not select.select([sys.stdin], [], [], 0.001)[0]:\n"
+        "    sample()\n"
+        "print(json.dumps({'max': mx, 'rows': rows[1:] or rows}), flush=True)\n"
+    )
+
+    def _bus_id(self):
         import torch
-        pynvml.nvmlInit()
-        try:
-            pr = torch.cuda.get_device_properties(self.gpu)
-            bus = f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0"
-            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
-        except Exception:
-            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
-
-    def _poll(self, pynvml, h):
-        get_reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons",
-                              getattr(pynvml, "nvmlDeviceGetCurrentClocksThrottleReasons", None))
-        mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
-        while not self.stop_flag:
-            try:
-                sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
-                rs = get_reasons(h) if get_reasons else 0
-                self.rows.append((sm, mx, rs))
-            except Exception:
-                pass
-            time.sleep(0.001)
+        pr = torch.cuda.get_device_properties(self.gpu)
+        return f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0"
 
     def start(self):
         try:
-            pynvml, h = self._nvml_handle()
-            self.stop_flag = False
-            self.thread = threading.Thread(target=self._poll, args=(pynvml, h), daemon=True)
-            self.thread.start()
-            time.sleep(0.01)
-            return
+            self.poller = subprocess.Popen([sys.executable, "-c", self.POLL, self._bus_id(), str(self.gpu)],
+                                           stdin=subprocess.PIPE, stdout=subprocess.PIPE,
+                                           stderr=subprocess.DEVNULL, text=True)
+            if self.poller.stdout.readline().strip() == "ready":
+                return
+            self.poller.kill()
         except Exception:
-            self.thread = None
+            pass
+        self.poller = None
         try:
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
@@ -115,17 +116,22 @@ class ClockSampler:
             self.proc = None
 
     def stop(self):
-        if self.thread is not None:
-            self.stop_flag = True
-            self.thread.join(timeout=5)
-            if not self.rows:
+        if self.poller is not None:
+            try:
+                out, _ = self.poller.communicate(input="stop\n", timeout=30)
+                d = json.loads(out.strip().splitlines()[-1])
+            except Exception:
+                self.poller.kill()
+                return None
+            rows = d["rows"]
+            if not rows:
                 return None
             # NVML reason bits: 0x4 sw power cap, 0x8 hw slowdown, 0x20 sw thermal, 0x40 hw thermal.
             bits = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown", 0x4: "sw_power_cap"}
-            sm = sorted(r[0] for r in self.rows)
-            reasons = sorted({name for r in self.rows for b, name in bits.items() if r[2] & b})
-            return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": self.rows[0][1], "reasons": reasons,
-                    "samples": len(self.rows), "source": "nvml"}
+            sm = sorted(r[0] for r in rows)
+            reasons = sorted({name for r in rows for b, name in bits.items() if r[1] & b})
+            return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": d["max"], "reasons": reasons,
+                    "samples": len(rows), "source": "nvml"}
         if self.proc is None:
             return None
         time.sleep(0.25)
