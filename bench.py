@@ -396,7 +396,9 @@ def run_ours(args, rank, world, local_rank):
     fused = {k: v for k, v in prof.items() if k.startswith("fused_nf4")}
     dom = max(fused, key=lambda k: fused[k][0])
     dom_ms = fused[dom][0] / fused[dom][1]
-    dom_flops = 2 * M * N * K + 2 * M * r * (N if dom.endswith("fwd") else K)
+    # Each fused launch also computes its rank-r intermediate (T = s X A in the
+    # forward, U = s dY B^T in the input gradient) besides the LoRA product.
+    dom_flops = 2 * M * N * K + 2 * M * r * (N + K)
     achieved = dom_flops / (dom_ms * 1e-3) / 1e12
     launches = sum(v[2] for v in prof.values())
     kernels = {k: {"ms_per_call": v[0] / v[1], "calls": v[1], "share": v[0] / sum(x[0] for x in prof.values())}

@@ -34,25 +34,22 @@ constexpr size_t kStatusBytes = 256;
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-// Workspace: [status word (256 B)][T pair: bf16 M x 2rp][U pair: bf16 M x 2rp]
-// [partial tiles of the rank-r products on the caller's stream][partial
-// tiles of dB, which runs on a second stream] and, when M <= kSmallMMax,
-// [small-M counters and partial tiles].
+// Workspace: [status word (256 B)][counters of the forward and input-gradient
+// GEMMs][T pair: bf16 M x 2rp][U pair: bf16 M x 2rp] and, when
+// M <= kSmallMMax, [small-M counters and partial tiles].
 struct WsLayout {
-  size_t t_off, u_off, rk_off, rk2_off, sm_off, total;
+  size_t cf_off, cd_off, t_off, u_off, sm_off, total;
 };
 
 WsLayout ws_layout(int64_t M, int64_t K, int64_t N, int r) {
   WsLayout w{};
   const size_t pair_bytes = round_up(static_cast<size_t>(M) * 2 * lora_pad(r) * 2, 256);
-  size_t rank_bytes = 0;
-  for (SkinnyKind k : {SkinnyKind::kXA, SkinnyKind::kDyBt, SkinnyKind::kTtDy, SkinnyKind::kXtU})
-    rank_bytes = std::max(rank_bytes, skinny_scratch_bytes(k, M, K, N, r));
-  w.t_off = kStatusBytes;
+  const size_t ctr_bytes = round_up(static_cast<size_t>(fused_ctr_ints(M)) * 4, 256);
+  w.cf_off = kStatusBytes;
+  w.cd_off = w.cf_off + ctr_bytes;
+  w.t_off = w.cd_off + ctr_bytes;
   w.u_off = w.t_off + pair_bytes;
-  w.rk_off = w.u_off + pair_bytes;
-  w.rk2_off = w.rk_off + round_up(rank_bytes, 256);
-  w.sm_off = w.rk2_off + round_up(skinny_scratch_bytes(SkinnyKind::kTtDy, M, K, N, r), 256);
+  w.sm_off = w.u_off + pair_bytes;
   w.total = w.sm_off + (M <= kSmallMMax ? round_up(small_m_workspace_bytes(M, N, r), 256) : 0);
   return w;
 }
@@ -128,33 +125,6 @@ struct ProfScope {
     on = false;
   }
 };
-
-// Second stream for the part of the backward that does not depend on U
-// (T pair -> dB), with the events that fork it from and join it to the
-// caller's stream.  One per host thread and device, so that calls from
-// different threads never share the fork/join events; created on first use
-// and kept for the life of the thread.
-struct AuxStream {
-  cudaStream_t st = nullptr;
-  cudaEvent_t fork = nullptr, join = nullptr;
-};
-constexpr int kMaxDevices = 64;
-thread_local AuxStream t_aux[kMaxDevices];
-
-cudaError_t aux_stream(AuxStream** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  AuxStream& a = t_aux[dev];
-  if (!a.st) {
-    if ((e = cudaStreamCreateWithFlags(&a.st, cudaStreamNonBlocking)) != cudaSuccess) return e;
-    if ((e = cudaEventCreateWithFlags(&a.fork, cudaEventDisableTiming)) != cudaSuccess) return e;
-    if ((e = cudaEventCreateWithFlags(&a.join, cudaEventDisableTiming)) != cudaSuccess) return e;
-  }
-  *out = &a;
-  return cudaSuccess;
-}
 
 }  // namespace
 
@@ -236,16 +206,12 @@ qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, int64_t K, int64_t N
     p0.done();
     return e == cudaSuccess ? QLORA_OK : cuda_fail(e);
   }
-  ProfScope p1(st, "lora_down_xa", 1);
-  float* rk = reinterpret_cast<float*>(ws + wl.rk_off);
-  cudaError_t e = launch_skinny(SkinnyKind::kXA, X, A, M, K, N, r, scale, SkinnyOut{T_save, Tpair}, rk, status, st);
-  p1.done();
-  if (e != cudaSuccess) return cuda_fail(e);
-  {
-    ProfScope p2(st, "fused_nf4_fwd", 1);
-    e = launch_fused_fwd(X, codes, absmax_q, absmax_scale, Tpair, B, M, K, N, r, Y, status, P, st);
-    p2.done();
-  }
+  // One launch: T = s X A (T_save and its pair) in the kernel's first units,
+  // then the output tiles.
+  ProfScope p2(st, "fused_nf4_fwd", 1);
+  const cudaError_t e = launch_fused_fwd(X, codes, absmax_q, absmax_scale, Tpair, B, M, K, N, r, Y, status, P, st, A,
+                                         T_save, scale, reinterpret_cast<int*>(ws + wl.cf_off));
+  p2.done();
   if (e != cudaSuccess) return cuda_fail(e);
   return QLORA_OK;
 }
@@ -273,46 +239,18 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   const Nf4Params& P = nf4_params();
 
-  // dB = T^T dY needs only T and dY, so it runs on a second stream next to
-  // the U -> dX -> dA chain (the rank-r products are latency-bound and two of
-  // them share the GPU well).  On the caller's stream every kernel comes right
-  // after the one whose output it reads (the kernels start early and wait for
-  // their predecessor only there).
-  AuxStream* aux = nullptr;
-  cudaError_t e = aux_stream(&aux);
-  if (e == cudaSuccess) e = cudaEventRecord(aux->fork, st);
-  if (e == cudaSuccess) e = cudaStreamWaitEvent(aux->st, aux->fork, 0);
+  // Two launches: the bf16 pair of T, then one GEMM launch that computes
+  // U = s dY B^T in its first units, the dX tiles, and dA = X^T U and
+  // dB = T^T dY in units that fill the SMs its last wave of tiles leaves idle.
+  ProfScope p1(st, "split_t_pair", 1);
+  cudaError_t e = launch_split_pair(T_save, M, r, Tpair, st);
+  p1.done();
   if (e != cudaSuccess) return cuda_fail(e);
-  float* rk = reinterpret_cast<float*>(ws + wl.rk_off);
-  float* rk2 = reinterpret_cast<float*>(ws + wl.rk2_off);
-  {
-    ProfScope p2(aux->st, "lora_db_ttdy", 2);
-    e = launch_split_pair(T_save, M, r, Tpair, aux->st);
-    if (e == cudaSuccess)
-      e = launch_skinny(SkinnyKind::kTtDy, dY, Tpair, M, K, N, r, 1.0f, SkinnyOut{dB, nullptr}, rk2, status, aux->st);
-    p2.done();
-  }
-  if (e == cudaSuccess) {
-    ProfScope p1(st, "lora_u_dybt", 1);
-    e = launch_skinny(SkinnyKind::kDyBt, dY, B, M, K, N, r, scale, SkinnyOut{nullptr, Upair}, rk, status, st);
-    p1.done();
-  }
-  if (e == cudaSuccess) {
-    ProfScope p3(st, "fused_nf4_dx", 1);
-    e = launch_fused_dx(dY, codes, absmax_q, absmax_scale, Upair, A, M, K, N, r, dX, status, P, st);
-    p3.done();
-  }
-  if (e == cudaSuccess) {
-    ProfScope p4(st, "lora_da_xtu", 1);
-    e = launch_skinny(SkinnyKind::kXtU, X, Upair, M, K, N, r, 1.0f, SkinnyOut{dA, nullptr}, rk, status, st);
-    p4.done();
-  }
-  // Join even after a failed launch, so the caller's stream never runs ahead
-  // of work already queued on the second stream.
-  cudaError_t ej = cudaEventRecord(aux->join, aux->st);
-  if (ej == cudaSuccess) ej = cudaStreamWaitEvent(st, aux->join, 0);
+  ProfScope p2(st, "fused_nf4_dx", 1);
+  e = launch_fused_dx(dY, codes, absmax_q, absmax_scale, Upair, A, M, K, N, r, dX, status, P, st, B, scale,
+                      reinterpret_cast<int*>(ws + wl.cd_off), X, Tpair, dA, dB);
+  p2.done();
   if (e != cudaSuccess) return cuda_fail(e);
-  if (ej != cudaSuccess) return cuda_fail(ej);
   return QLORA_OK;
 }
 

@@ -7,6 +7,25 @@
 //   forward         Y  = X  W'^T + [T_hi | T_lo] [B ; B]      (B operand K-major)
 //   input gradient  dX = dY W'   + [U_hi | U_lo] [A^T ; A^T]  (B operand MN-major)
 //
+// The rank-r intermediate the LoRA stages read (T = s X A in the forward,
+// U = s dY B^T in the input gradient) is computed by the same kernel: the
+// first tickets of the grid are "rank units", one per 512-row block, that
+// stream the same activation rows through the same pipeline against a
+// 64-column slice of the adapter matrix per CTA (N = 128 across the pair),
+// write the float32 result and its bf16 pair, and raise that block's ready
+// count.  Output tiles wait for the count only before their LoRA stages, so
+// the rank units run in the time the grid's last wave would leave SMs idle,
+// and no separate launch stands between the inputs and the GEMM.
+//
+// The input-gradient launch also forms the adapter gradients in "tail
+// units": dA = X^T U and dB^T = dY^T T, each unit 512 rows of the result
+// reduced over all M tokens in TMEM (A operand MN-major: activation columns;
+// B operand the [hi | lo] pair, N = 2rp across the pair, the halves added in
+// the epilogue).  Tickets go out as: rank units; tiles for the rest of the
+// first wave; as many tail units as there are rank units (taken by the pairs
+// that finish the shorter rank units first); the remaining tiles; the
+// remaining tail units (short jobs that fill the last wave's idle SMs).
+//
 // Two CTAs of a cluster compute one 512 x 256 output tile.  Each CTA holds
 // 2 x 128 rows of the activation tile (one 128-row half of each of two
 // M = 256 pair-MMAs) and decodes its own 128-row half of the weight tile; the
@@ -45,6 +64,22 @@ constexpr int kThreads = 384;
 constexpr int kDecWarps = 4;      // decoder warps per stage (warps 4-7 even stages, 8-11 odd)
 
 struct PairArgs {
+  int units;        // CTA pairs in the grid
+  int tiles_n;      // output tiles along the columns
+  // Rank units (one per 512-row block) ahead of the output tiles, or 0 when
+  // the bf16 pair comes from the previous kernel in the stream.
+  int r_units;
+  int* ctr;         // [ticket, done, ready count per row block]; null: units by block index
+  int r;            // adapter rank
+  float scale;      // LoRA scale s, applied to the rank-r intermediate
+  float* r_f32;     // float32 intermediate [rows x r] (forward T) or null
+  uint16_t* r_pair; // bf16 pair of the intermediate, read by the LoRA stages
+  // Tail units (input gradient only): da_units of dA then dB ones.  The first
+  // t_first go out after the first `early` tiles, the rest after all tiles.
+  int t_units, da_units, early, t_first;
+  int nmb;          // 64-row blocks of M (reduction depth of a tail unit)
+  float* dA;        // [K x r]
+  float* dB;        // [r x N]
   int nkb;          // main 64-deep stages
   int lora_kb;      // LoRA stages (hi and lo halves of the pair)
   int lora_mod;     // rp: LoRA stage lk reads the adapter at (64*lk) mod rp
@@ -57,6 +92,12 @@ struct PairArgs {
   int abs_tma;             // dX: 8-bit constant codes by TMA
   int* status;
   Nf4Params nf4;
+};
+
+// Tensor maps of the tail units: activation columns (64 x 64 boxes) and the
+// bf16 pairs they are reduced against.
+struct TailMaps {
+  CUtensorMap a_da, b_da, a_db, b_db;
 };
 
 template <bool MNB>
@@ -75,7 +116,8 @@ struct PairSmem {
   static constexpr int kNumBars = 4 * kStages + 1;
   static constexpr int offSlot = offBar + kNumBars * 8;
   static constexpr int offAbort = offSlot + 4;
-  static constexpr int kTotal = offAbort + 4;
+  static constexpr int offUnit = offAbort + 4;
+  static constexpr int kTotal = offUnit + 4;
   static constexpr int kDynamic = kTotal + 1024;
 };
 
@@ -99,6 +141,11 @@ __device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap* map, uint32_
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(mbar_cluster), "r"(x), "r"(y)
       : "memory");
+}
+__device__ __forceinline__ int ld_cluster_s32(uint32_t addr) {
+  int v;
+  asm volatile("ld.shared::cluster.b32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
 }
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t mbar_cluster) {
   asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(mbar_cluster) : "memory");
@@ -136,9 +183,11 @@ template <bool MNB>
 __global__ void __launch_bounds__(kThreads, 1)
     fused_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmC,
                       const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
-                      const __grid_constant__ CUtensorMap tmAbs, const PairArgs args) {
+                      const __grid_constant__ CUtensorMap tmAbs, const __grid_constant__ CUtensorMap tmR,
+                      const __grid_constant__ TailMaps tm, const PairArgs args) {
   using L = PairSmem<MNB>;
   constexpr uint32_t kTmemCols = 512;  // two 128 x 256 fp32 accumulators
+  constexpr int kRankB = 64 * kDepth * 2;  // a rank unit's adapter tile per CTA and stage
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -154,13 +203,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* acc_full = decoded + kStages;                          // local: accumulators ready
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::offSlot);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::offAbort);
+  int* unit_slot = reinterpret_cast<int*>(smem + L::offUnit);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();  // 0 = leader
-  const int tile_n = blockIdx.x >> 1;
-  const int tile_m = blockIdx.y;
-  const int total = args.nkb + args.lora_kb;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -178,18 +225,44 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmC);
     tma_prefetch_desc(&tmA2);
     tma_prefetch_desc(&tmB2);
+    if (args.r_units) tma_prefetch_desc(&tmR);
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, kTmemCols);
     tmem_relinquish_pair();
   }
+  if (args.ctr) {
+    // Units by ticket, so that the rank units (the first tickets) have started
+    // before any tile can wait for them.  All inputs may come from the
+    // previous kernel in the stream: wait for it before the first load.
+    griddep_wait();
+    if (threadIdx.x == 0 && rank == 0) *unit_slot = atomicAdd(args.ctr, 1);
+  }
   tc_fence_before();
   __syncthreads();
-  cluster_sync_all();  // the leader's barriers exist before the peer signals them
+  cluster_sync_all();  // the leader's barriers (and ticket) exist before the peer uses them
   tc_fence_after();
   const uint32_t tmem_acc = *tmem_slot;
-  // The previous kernel in the stream produces only the LoRA intermediate
-  // (T or U pair), read in the last stages: everything else may start now.
+  int unit = static_cast<int>(blockIdx.x >> 1);
+  if (args.ctr) unit = rank == 0 ? *unit_slot : ld_cluster_s32(map_rank(unit_slot, 0));
+  // Ticket order: rank units; tiles [0, early); tail units [0, t_first);
+  // the other tiles; the other tail units.
+  const bool runit = unit < args.r_units;
+  const int v = unit - args.r_units;
+  const int ntiles = args.units - args.r_units - args.t_units;
+  int tile = 0, tj = -1;
+  if (!runit) {
+    if (v < args.early) tile = v;
+    else if (v < args.early + args.t_first) tj = v - args.early;
+    else if (v < ntiles + args.t_first) tile = v - args.t_first;
+    else tj = v - ntiles;
+  }
+  const bool tunit = tj >= 0;
+  const int tile_m = runit ? unit : tile / args.tiles_n;
+  const int tile_n = tile % args.tiles_n;
+  const int total = runit ? args.nkb : (tunit ? args.nmb : args.nkb + args.lora_kb);
+  // Without rank units the previous kernel produces only the LoRA
+  // intermediate, read in the last stages: everything else may start now.
   griddep_launch_dependents();
 
   if (warp == 0) {
@@ -205,11 +278,46 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* a_dst = sA + s * L::kA;
         uint8_t* b_dst = sB + s * L::kB;
         const int row0 = tile_m * kPairRows + static_cast<int>(rank) * 128;
+        if (tunit) {
+          // 64 tokens per stage: this CTA's 2 x 128 result rows of the
+          // activation (four 64-column boxes) and its rp columns of the pair.
+          const bool is_da = tj < args.da_units;
+          if (i == 0 && is_da) {
+            bool ok = true;
+            for (int m = 0; m < args.r_units && ok; ++m) ok = wait_count(args.ctr + 2 + m, 2, ctx);
+            if (!ok) break;
+            fence_proxy_async_global();  // U is written by this launch's rank units
+          }
+          const CUtensorMap* am = is_da ? &tm.a_da : &tm.a_db;
+          const CUtensorMap* bm = is_da ? &tm.b_da : &tm.b_db;
+          const int c0 = (is_da ? tj : tj - args.da_units) * kPairRows + static_cast<int>(rank) * 128;
+          const int nb = args.lora_mod / 64;
+          if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * L::kA + 2 * nb * 8192);
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int a = 0; a < 2; ++a)
+              tma_load_2d_pair(am, full_leader, a_dst + h * 16384 + a * 8192, c0 + h * 256 + a * 64, i * kDepth);
+          for (int b = 0; b < nb; ++b)
+            tma_load_2d_pair(bm, full_leader, b_dst + b * 8192, static_cast<int>(rank) * args.lora_mod + b * 64,
+                             i * kDepth);
+          ++issued;
+          continue;
+        }
         if (i < args.nkb) {
           const int kb = i;
-          if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * L::kA);
+          if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * L::kA + (runit ? 2 * kRankB : 0));
           tma_load_2d_pair(&tmA, full_leader, a_dst, kb * kDepth, row0);
           tma_load_2d_pair(&tmA, full_leader, a_dst + 16384, kb * kDepth, row0 + 256);
+          if (runit) {
+            // This CTA's 64 adapter columns: forward A[K, r] rows of block kb
+            // (MN-major B operand), input gradient B[r, N] columns of block kb
+            // (K-major).  Columns past r read as zeros.
+            if (!MNB) tma_load_2d_pair(&tmR, full_leader, b_dst, static_cast<int>(rank) * 64, kb * kDepth);
+            else tma_load_2d_pair(&tmR, full_leader, b_dst, kb * kDepth, static_cast<int>(rank) * 64);
+            ++issued;
+            continue;
+          }
           const bool abs_tma = MNB && args.abs_tma;
           mbar_arrive_expect_tx(&cfull[s], L::kC + (abs_tma ? 1024 : 0));
           if (!MNB) {
@@ -225,7 +333,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           const int lk = i - args.nkb;
           const int lb = (lk * kDepth) % args.lora_mod;
-          if (lk == 0) griddep_wait();  // the pair is the previous kernel's output
+          if (lk == 0) {
+            if (args.ctr) {
+              // the pair is written by this row block's rank unit
+              if (!wait_count(args.ctr + 2 + tile_m, 2, ctx)) break;
+              fence_proxy_async_global();
+            } else {
+              griddep_wait();  // the pair is the previous kernel's output
+            }
+          }
           if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * (L::kA + L::kB));
           tma_load_2d_pair(&tmA2, full_leader, a_dst, lk * kDepth, row0);
           tma_load_2d_pair(&tmA2, full_leader, a_dst + 16384, lk * kDepth, row0 + 256);
@@ -246,8 +362,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t t0 = globaltimer_ns();
           const int s = i % kStages;
           const uint32_t ph = (i / kStages) & 1;
+          const bool codes = i < args.nkb && !runit && !tunit;  // only these stages load codes
           while (globaltimer_ns() - t0 < kWaitTimeoutNs &&
-                 !(mbar_try_wait(&cfull[s], ph) && (rank != 0 || mbar_try_wait(&full[s], ph)))) {
+                 !((!codes || mbar_try_wait(&cfull[s], ph)) && (rank != 0 || mbar_try_wait(&full[s], ph)))) {
           }
         }
       }
@@ -264,25 +381,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       // M = 256 across the pair, N = 256 (each CTA supplies 128 columns of B).
       const uint32_t idesc_main = idesc_bf16_f32(256, 256, false, MNB);
       const uint32_t idesc_lora = idesc_bf16_f32(256, 256, false, !MNB);
+      const uint32_t idesc_unit = idesc_bf16_f32(256, 128, false, !MNB);
+      const uint32_t idesc_tail = idesc_bf16_f32(256, 2 * args.lora_mod, true, true);
       const uint32_t d = tmem_acc + h * 256;
       bool ok = true;
       for (int i = 0; i < total && ok; ++i) {
         const int s = i % kStages;
         const uint32_t ph = (i / kStages) & 1;
         const bool main_stage = i < args.nkb;
+        const bool dec_stage = main_stage && !runit && !tunit;  // B is the decoded weight
         if (!mbar_wait(&full[s], ph, ctx)) { ok = false; break; }
-        if (main_stage && !mbar_wait(&decoded[s], ph, ctx)) { ok = false; break; }
+        if (dec_stage && !mbar_wait(&decoded[s], ph, ctx)) { ok = false; break; }
         tc_fence_after();
         const uint32_t a_base = smem_u32(sA + s * L::kA) + h * 16384;
         const uint32_t b_base = smem_u32(sB + s * L::kB);
-        const bool b_mn = main_stage ? MNB : !MNB;
+        // The B operand is the decoded weight in main stages of output tiles
+        // and an adapter matrix or pair otherwise; only tail units read A
+        // MN-major.
+        const bool b_mn = tunit || (dec_stage ? MNB : !MNB);
+        const uint32_t idesc = tunit ? idesc_tail : (runit ? idesc_unit : (main_stage ? idesc_main : idesc_lora));
 #pragma unroll
         for (int kk = 0; kk < kDepth / 16; ++kk) {
           const uint64_t bdesc = b_mn ? smem_desc_sw128(b_base + kk * 2048, 8192, 1024)
                                       : smem_desc_sw128(b_base + kk * 32, 16, 1024);
-          const uint32_t idesc = main_stage ? idesc_main : idesc_lora;
+          const uint64_t adesc = tunit ? smem_desc_sw128(a_base + kk * 2048, 8192, 1024)
+                                       : smem_desc_sw128(a_base + kk * 32, 16, 1024);
           const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
-          umma_pair(d, smem_desc_sw128(a_base + kk * 32, 16, 1024), bdesc, idesc, acc);
+          umma_pair(d, adesc, bdesc, idesc, acc);
         }
         umma_commit_pair(&empty[s]);
       }
@@ -299,7 +424,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       lvl2[threadIdx.x - 128] = level2_value(threadIdx.x - 128);
       asm volatile("bar.sync 1, 256;" ::: "memory");
       const int64_t blocks_per_row = args.w_cols / 64;
-      if (!MNB) {
+      if (runit || tunit) {
+        // rank and tail units read no weight
+      } else if (!MNB) {
         // Thread d decodes weight row n (this CTA's half), one block per stage.
         const int64_t n = static_cast<int64_t>(tile_n) * kPairCols + rank * 128 + d;
         const bool row_ok = n < args.w_rows;
@@ -416,9 +543,84 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int h = (warp - 4) >> 2;  // accumulator (first or second M = 256 MMA)
       const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(acc_full, 0, ctx));
       tc_fence_after();
-      if (ok) {
-        const int row = tile_m * kPairRows + h * 256 + static_cast<int>(rank) * 128 + q * 32 + lane;
-        const uint32_t t_row = tmem_acc + (static_cast<uint32_t>(q * 32) << 16) + h * 256;
+      const int row = tile_m * kPairRows + h * 256 + static_cast<int>(rank) * 128 + q * 32 + lane;
+      const uint32_t t_row = tmem_acc + (static_cast<uint32_t>(q * 32) << 16) + h * 256;
+      if (ok && runit) {
+        // v = s * acc in float32 (the forward keeps it as T); the pair holds
+        // hi = bf16(v) in columns [0, rp) and lo = bf16(v - hi) in [rp, 2rp),
+        // zero past r.
+        const int rp = args.lora_mod;
+#pragma unroll 1
+        for (int cc = 0; cc < rp / 32; ++cc) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(t_row + cc * 32, v);
+          tmem_wait_ld();
+          if (row < args.rows) {
+            uint16_t* pr = args.r_pair + static_cast<int64_t>(row) * 2 * rp;
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              const int c0 = cc * 32 + g * 8;
+              float sv[8];
+              uint32_t hi[4], lo[4];
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                sv[e] = (c0 + e < args.r) ? __fmul_rn(args.scale, __uint_as_float(v[g * 8 + e])) : 0.0f;
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const __nv_bfloat16 h0 = __float2bfloat16_rn(sv[2 * e]);
+                const __nv_bfloat16 h1 = __float2bfloat16_rn(sv[2 * e + 1]);
+                const __nv_bfloat16 l0 = __float2bfloat16_rn(__fsub_rn(sv[2 * e], __bfloat162float(h0)));
+                const __nv_bfloat16 l1 = __float2bfloat16_rn(__fsub_rn(sv[2 * e + 1], __bfloat162float(h1)));
+                hi[e] = __bfloat16_as_ushort(h0) | (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
+                lo[e] = __bfloat16_as_ushort(l0) | (static_cast<uint32_t>(__bfloat16_as_ushort(l1)) << 16);
+              }
+              *reinterpret_cast<uint4*>(pr + c0) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+              *reinterpret_cast<uint4*>(pr + rp + c0) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+              if (args.r_f32 && c0 < args.r) {
+                float* tf = args.r_f32 + static_cast<int64_t>(row) * args.r + c0;
+                *reinterpret_cast<float4*>(tf) = make_float4(sv[0], sv[1], sv[2], sv[3]);
+                *reinterpret_cast<float4*>(tf + 4) = make_float4(sv[4], sv[5], sv[6], sv[7]);
+              }
+            }
+          }
+        }
+      } else if (ok && tunit) {
+        // Result rows (k of dA, n of dB) in lanes; columns [0, rp) hold the
+        // product with the hi half of the pair, [rp, 2rp) with the lo half.
+        const int rp = args.lora_mod;
+        const bool is_da = tj < args.da_units;
+        const int rrow = (is_da ? tj : tj - args.da_units) * kPairRows + h * 256 + static_cast<int>(rank) * 128 +
+                         q * 32 + lane;
+        const bool in = rrow < (is_da ? args.w_cols : args.w_rows);
+#pragma unroll 1
+        for (int cc = 0; cc < rp / 32; ++cc) {
+          uint32_t vh[32], vl[32];
+          tmem_ld_32x32b_x32(t_row + cc * 32, vh);
+          tmem_ld_32x32b_x32(t_row + rp + cc * 32, vl);
+          tmem_wait_ld();
+          if (in) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 4) {
+              const int j = cc * 32 + e;
+              if (j < args.r) {
+                const float4 o = make_float4(__fadd_rn(__uint_as_float(vh[e]), __uint_as_float(vl[e])),
+                                             __fadd_rn(__uint_as_float(vh[e + 1]), __uint_as_float(vl[e + 1])),
+                                             __fadd_rn(__uint_as_float(vh[e + 2]), __uint_as_float(vl[e + 2])),
+                                             __fadd_rn(__uint_as_float(vh[e + 3]), __uint_as_float(vl[e + 3])));
+                if (is_da) {
+                  *reinterpret_cast<float4*>(args.dA + static_cast<int64_t>(rrow) * args.r + j) = o;
+                } else {
+                  float* col = args.dB + static_cast<int64_t>(j) * args.w_rows + rrow;
+                  col[0] = o.x;
+                  col[args.w_rows] = o.y;
+                  col[2 * args.w_rows] = o.z;
+                  col[3 * args.w_rows] = o.w;
+                }
+              }
+            }
+          }
+        }
+      } else if (ok) {
 #pragma unroll 1
         for (int cc = 0; cc < kPairCols / 32; ++cc) {
           uint32_t v[32];
@@ -441,6 +643,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      if (runit) {
+        // Publish this CTA's half of the row block: stores visible to other
+        // CTAs' TMA loads, then one count per CTA (the tiles wait for 2).
+        fence_proxy_async_global();
+        __threadfence();
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+        if (threadIdx.x == 128) atomicAdd(args.ctr + 2 + tile_m, 1);
+      }
     }
   }
 
@@ -451,18 +661,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc_pair(tmem_acc, kTmemCols);
   }
+  if (args.ctr && threadIdx.x == 0 && rank == 0) {
+    // The last pair to finish returns the counters to zero: every pair has
+    // taken its ticket and is past its last look at a ready count.
+    __threadfence();
+    if (atomicAdd(args.ctr + 1, 1) == args.units - 1) {
+      for (int m = 0; m < args.r_units; ++m) args.ctr[2 + m] = 0;
+      args.ctr[0] = 0;
+      args.ctr[1] = 0;
+      __threadfence();
+    }
+  }
 }
 
 template <bool MNB>
 cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& c, const CUtensorMap& a2, const CUtensorMap& b2,
-                        const CUtensorMap& abs, const PairArgs& args, int tiles_n, int tiles_m, cudaStream_t stream) {
+                        const CUtensorMap& abs, const CUtensorMap& rmap, const TailMaps& tmaps, const PairArgs& args,
+                        cudaStream_t stream) {
   using L = PairSmem<MNB>;
   static_assert(L::kDynamic <= 232448, "shared memory budget");
   auto kern = fused_pair_kernel<MNB>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kDynamic);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(2 * tiles_n), static_cast<unsigned>(tiles_m), 1);
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * args.units), 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = L::kDynamic;
   cfg.stream = stream;
@@ -474,23 +696,59 @@ cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& c, const CUtens
   attr[1] = pdl_attribute();
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, kern, a, c, a2, b2, abs, args);
+  return cudaLaunchKernelEx(&cfg, kern, a, c, a2, b2, abs, rmap, tmaps, args);
+}
+
+// Unit count and rank-unit fields shared by both directions.
+void plan_units(PairArgs& args, int64_t M, int64_t cols, int r, float scale, int* ctr, float* r_f32,
+                uint16_t* r_pair) {
+  const int tiles_n = static_cast<int>((cols + kPairCols - 1) / kPairCols);
+  const int tiles_m = static_cast<int>((M + kPairRows - 1) / kPairRows);
+  args.tiles_n = tiles_n;
+  args.r_units = ctr ? tiles_m : 0;
+  args.units = tiles_m * tiles_n + args.r_units;
+  args.ctr = ctr;
+  args.r = r;
+  args.scale = scale;
+  args.r_f32 = r_f32;
+  args.r_pair = r_pair;
+  args.early = tiles_m * tiles_n;
+}
+
+// CTA pairs resident at once (one 1-CTA-per-SM pair per two SMs).
+int resident_pairs() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 1;
+  return std::max(1, sms / 2);
 }
 
 }  // namespace
 
+int fused_ctr_ints(int64_t M) { return 2 + static_cast<int>((M + kPairRows - 1) / kPairRows); }
+
 cudaError_t launch_fused_fwd(const uint16_t* X, const uint8_t* codes, const uint8_t* absmax_q,
-                             const float* absmax_scale, const uint16_t* Tpair, const uint16_t* B, int64_t M, int64_t K,
-                             int64_t N, int r, uint16_t* Y, int* status, const Nf4Params& P, cudaStream_t stream) {
+                             const float* absmax_scale, uint16_t* Tpair, const uint16_t* B, int64_t M, int64_t K,
+                             int64_t N, int r, uint16_t* Y, int* status, const Nf4Params& P, cudaStream_t stream,
+                             const uint16_t* A, float* T_save, float scale, int* ctr) {
   const int rp = lora_pad(r);
-  CUtensorMap mX, mC, mT, mB;
+  CUtensorMap mX, mC, mT, mB, mR;
   if (!make_map_2d(&mX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, K * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map_2d(&mC, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, K / 2, N, K / 2, 32, 128, CU_TENSOR_MAP_SWIZZLE_32B) ||
       !make_map_2d(&mT, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Tpair, 2 * rp, M, static_cast<int64_t>(rp) * 4, 64, 128,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map_2d(&mB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, B, N, r, N * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
+  mR = mB;
+  if (ctr) {
+    // A [K, r]: 64 reduction rows x 64 adapter columns per CTA and stage
+    if (!A || !T_save ||
+        !make_map_2d(&mR, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, r, K, static_cast<int64_t>(r) * 2, 64, 64,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+  }
   PairArgs args{};
+  plan_units(args, M, N, r, scale, ctr, T_save, Tpair);
   args.nkb = static_cast<int>(K / 64);
   args.lora_kb = 2 * rp / 64;
   args.lora_mod = rp;
@@ -505,16 +763,17 @@ cudaError_t launch_fused_fwd(const uint16_t* X, const uint8_t* codes, const uint
   args.abs_tma = 0;
   args.status = status;
   args.nf4 = P;
-  const int tiles_n = static_cast<int>((N + kPairCols - 1) / kPairCols);
-  const int tiles_m = static_cast<int>((M + kPairRows - 1) / kPairRows);
-  return launch_pair<false>(mX, mC, mT, mB, mB, args, tiles_n, tiles_m, stream);
+  const TailMaps none{mB, mB, mB, mB};
+  return launch_pair<false>(mX, mC, mT, mB, mB, mR, none, args, stream);
 }
 
 cudaError_t launch_fused_dx(const uint16_t* dY, const uint8_t* codes, const uint8_t* absmax_q,
-                            const float* absmax_scale, const uint16_t* Upair, const uint16_t* A, int64_t M, int64_t K,
-                            int64_t N, int r, uint16_t* dX, int* status, const Nf4Params& P, cudaStream_t stream) {
+                            const float* absmax_scale, uint16_t* Upair, const uint16_t* A, int64_t M, int64_t K,
+                            int64_t N, int r, uint16_t* dX, int* status, const Nf4Params& P, cudaStream_t stream,
+                            const uint16_t* B, float scale, int* ctr, const uint16_t* X, const uint16_t* Tpair,
+                            float* dA, float* dB) {
   const int rp = lora_pad(r);
-  CUtensorMap mD, mC, mU, mA;
+  CUtensorMap mD, mC, mU, mA, mR;
   if (!make_map_2d(&mD, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dY, N, M, N * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map_2d(&mC, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, K / 2, N, K / 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_64B) ||
       !make_map_2d(&mU, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Upair, 2 * rp, M, static_cast<int64_t>(rp) * 4, 64, 128,
@@ -522,11 +781,39 @@ cudaError_t launch_fused_dx(const uint16_t* dY, const uint8_t* codes, const uint
       !make_map_2d(&mA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, r, K, static_cast<int64_t>(r) * 2, 64, 128,
                    CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
+  mR = mA;
+  if (ctr) {
+    // B [r, N]: 64 adapter rows x 64 reduction columns per CTA and stage
+    if (!B || !make_map_2d(&mR, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, B, N, r, N * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+  }
   CUtensorMap mAbs = mA;
   const bool abs_tma = (K % 1024 == 0) &&
                        make_map_2d(&mAbs, CU_TENSOR_MAP_DATA_TYPE_UINT8, absmax_q, K / 64, N, K / 64, 16, 64,
                                    CU_TENSOR_MAP_SWIZZLE_NONE);
   PairArgs args{};
+  plan_units(args, M, K, r, scale, ctr, nullptr, Upair);
+  TailMaps tails{mA, mA, mA, mA};
+  if (ctr && dA && dB) {
+    // dA = X^T U and dB^T = dY^T T: 64 tokens x 64 result rows per box
+    const int64_t ps = static_cast<int64_t>(rp) * 4;
+    if (!X || !Tpair ||
+        !make_map_2d(&tails.a_da, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, K * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_2d(&tails.b_da, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Upair, 2 * rp, M, ps, 64, 64,
+                     CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_2d(&tails.a_db, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dY, N, M, N * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_2d(&tails.b_db, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Tpair, 2 * rp, M, ps, 64, 64,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+    args.da_units = static_cast<int>((K + kPairRows - 1) / kPairRows);
+    args.t_units = args.da_units + static_cast<int>((N + kPairRows - 1) / kPairRows);
+    args.early = std::min(args.early, std::max(0, resident_pairs() - args.r_units));
+    args.t_first = std::min(args.t_units, args.r_units);
+    args.units += args.t_units;
+    args.nmb = static_cast<int>((M + 63) / 64);
+    args.dA = dA;
+    args.dB = dB;
+  }
   args.nkb = static_cast<int>((N + 63) / 64);
   args.lora_kb = 2 * rp / 64;
   args.lora_mod = rp;
@@ -541,9 +828,7 @@ cudaError_t launch_fused_dx(const uint16_t* dY, const uint8_t* codes, const uint
   args.abs_tma = abs_tma ? 1 : 0;
   args.status = status;
   args.nf4 = P;
-  const int tiles_n = static_cast<int>((K + kPairCols - 1) / kPairCols);
-  const int tiles_m = static_cast<int>((M + kPairRows - 1) / kPairRows);
-  return launch_pair<true>(mD, mC, mU, mA, mAbs, args, tiles_n, tiles_m, stream);
+  return launch_pair<true>(mD, mC, mU, mA, mAbs, mR, tails, args, stream);
 }
 
 }  // namespace qlora

@@ -34,14 +34,30 @@ cudaError_t launch_dequantize_nf4(const uint8_t* codes, const uint8_t* absmax_q,
 inline int lora_pad(int r) { return (r + 63) / 64 * 64; }
 
 // Fused dequant-GEMM, forward: Y[M,N] = X[M,K] W'[N,K]^T + (T_hi + T_lo)[M,r] B[r,N].
+// With `ctr` (fused_ctr_ints(M) ints, zero, left at zero) the kernel also
+// computes T = s X A itself (T_save float32 and the pair in Tpair) in units
+// that run ahead of the output tiles; with ctr == nullptr Tpair must be the
+// output of the previous kernel in the stream (A, T_save, scale unused).
 cudaError_t launch_fused_fwd(const uint16_t* X, const uint8_t* codes, const uint8_t* absmax_q,
-                             const float* absmax_scale, const uint16_t* Tpair, const uint16_t* B, int64_t M, int64_t K,
-                             int64_t N, int r, uint16_t* Y, int* status, const Nf4Params& P, cudaStream_t stream);
+                             const float* absmax_scale, uint16_t* Tpair, const uint16_t* B, int64_t M, int64_t K,
+                             int64_t N, int r, uint16_t* Y, int* status, const Nf4Params& P, cudaStream_t stream,
+                             const uint16_t* A = nullptr, float* T_save = nullptr, float scale = 0.0f,
+                             int* ctr = nullptr);
 
 // Fused dequant-GEMM, input gradient: dX[M,K] = dY[M,N] W'[N,K] + (U_hi + U_lo)[M,r] A[K,r]^T.
+// With `ctr` the kernel also computes U = s dY B^T (its pair in Upair) the
+// same way, and, when dA and dB are given, dA = X^T U and dB = T^T dY
+// (Tpair: the bf16 pair of T, written before this launch); with
+// ctr == nullptr Upair comes from the previous kernel.
 cudaError_t launch_fused_dx(const uint16_t* dY, const uint8_t* codes, const uint8_t* absmax_q,
-                            const float* absmax_scale, const uint16_t* Upair, const uint16_t* A, int64_t M, int64_t K,
-                            int64_t N, int r, uint16_t* dX, int* status, const Nf4Params& P, cudaStream_t stream);
+                            const float* absmax_scale, uint16_t* Upair, const uint16_t* A, int64_t M, int64_t K,
+                            int64_t N, int r, uint16_t* dX, int* status, const Nf4Params& P, cudaStream_t stream,
+                            const uint16_t* B = nullptr, float scale = 0.0f, int* ctr = nullptr,
+                            const uint16_t* X = nullptr, const uint16_t* Tpair = nullptr, float* dA = nullptr,
+                            float* dB = nullptr);
+
+// Counter ints one fused launch with rank units needs for M rows.
+int fused_ctr_ints(int64_t M);
 
 // Small-M forward (M <= kSmallMMax tokens): the whole forward (T = s X A, its
 // pair and Y) in one launch of a persistent weight-streaming kernel.

@@ -90,6 +90,34 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
   }
 }
 
+// ---------------------------------------------------------------- flags in global memory
+// A CTA that publishes data for other CTAs' TMA loads stores it, runs
+// fence_proxy_async_global + __threadfence, then raises a counter; the reader
+// acquires the counter and runs fence_proxy_async_global before its loads.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+__device__ __forceinline__ int ld_acquire(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+// Bounded wait until *p >= need.
+__device__ __forceinline__ bool wait_count(const int* p, int need, const WaitCtx& ctx) {
+  if (ld_acquire(p) >= need) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    __nanosleep(128);
+    if (ld_acquire(p) >= need) return true;
+    if (*ctx.abort_flag) return false;
+    if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+      *ctx.abort_flag = 1;
+      if (ctx.status) atomicCAS(ctx.status, 0, 0x100 + ctx.site);
+      return false;
+    }
+  }
+}
+
 // ---------------------------------------------------------------- dependent launch
 // Kernels launched with programmatic stream serialization may start while
 // their predecessor in the stream is still running.  griddep_wait blocks the

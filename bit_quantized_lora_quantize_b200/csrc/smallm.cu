@@ -169,15 +169,6 @@ __host__ __device__ __forceinline__ int64_t t_cum(int c, const SmallMArgs& a) {
 __host__ __device__ __forceinline__ int64_t pos_start(int c, const SmallMArgs& a) {
   return static_cast<int64_t>(c) * a.W / a.grid;
 }
-__device__ __forceinline__ void fence_proxy_async_global() {
-  asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-__device__ __forceinline__ int ld_acquire(const int* p) {
-  int v;
-  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
 // Bounded wait until the T pair is complete.
 __device__ __forceinline__ bool wait_t_ready(const SmallMArgs& a, const WaitCtx& ctx) {
   if (ld_acquire(a.t_ready) >= kReadyCount) return true;

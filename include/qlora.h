@@ -147,14 +147,10 @@ QLORA_API qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, int64_t K,
  *   T_save         in   float[M x r] as written by qlora_linear_fwd
  *   dX             out  bf16[M x K]
  *   dA, dB         out  float (overwritten, not accumulated)
- * Same supported shapes and workspace rule as qlora_linear_fwd.  The
- * reductions over M are split across thread blocks and summed in a fixed
- * order: results are bit-reproducible run to run.
- * dB runs on a second stream that this library keeps per host thread and
- * device, forked from `stream` at the start of the call and joined back into
- * it before the call returns (event record + stream wait), so all work is
- * ordered after what `stream` held before the call and before what it gets
- * after.  Inside a stream capture the fork and join become graph edges.
+ * Same supported shapes and workspace rule as qlora_linear_fwd.  Results
+ * are bit-reproducible run to run.
+ * Each reduction (U over N; dA, dB over M) is a single float32 chain in
+ * tensor-core accumulators, in a fixed order.
  */
 QLORA_API qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float* T_save, int64_t M, int64_t K,
                               int64_t N, const uint8_t* codes, const uint8_t* absmax_q, const float* absmax_scale,

@@ -81,6 +81,31 @@ def test_small_m_repeated_calls_are_identical():
     assert_close_rms(f64(outs[0]), Y, "Y")
 
 
+def test_repeated_calls_on_one_workspace_are_identical():
+    """The GEMM launches hand out work by ticket and publish T and U per
+    512-row block through counters in the workspace that each launch returns
+    to zero: three forward + backward passes on one workspace give the same
+    bits (a counter left behind would stall the next call into a timeout)."""
+    case = synthetic.linear_case(1100, 512, 640, 64, 0.25, seed=31)
+    Wp = q.qlora_quantize_nf4(case.W.to(DEV))
+    X, A, B, dY = (t.to(DEV) for t in (case.X, case.A, case.B, case.dY))
+    ws = q.new_workspace(case.M, case.K, case.N, case.r, DEV)
+    runs = []
+    for _ in range(3):
+        Y, T = q.qlora_linear_fwd(X, Wp, A, B, case.scale, workspace=ws)
+        runs.append((Y, T) + tuple(q.qlora_linear_bwd(dY, X, T, Wp, A, B, case.scale, workspace=ws)))
+    assert q.qlora_check_status(ws) == 0
+    for k in range(5):
+        assert torch.equal(runs[0][k], runs[1][k]) and torch.equal(runs[0][k], runs[2][k]), k
+    check_full(case, dict(zip(("Y", "T", "dX", "dA", "dB"), runs[0])))
+
+
+def test_many_row_blocks_few_column_tiles():
+    """16 row blocks and one column tile: as many rank units as output tiles."""
+    case = synthetic.linear_case(8000, 256, 200, 72, 0.5, seed=33)
+    check_full(case, run_gpu(case))
+
+
 def test_special_cases_exact():
     base = synthetic.linear_case(192, 256, 320, 16, 1.0, seed=21)
     # B = 0: no gradient reaches A, bit-exactly; Y is the frozen product.
