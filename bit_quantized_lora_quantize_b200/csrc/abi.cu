@@ -239,16 +239,12 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   const Nf4Params& P = nf4_params();
 
-  // Two launches: the bf16 pair of T, then one GEMM launch that computes
-  // U = s dY B^T in its first units, the dX tiles, and dA = X^T U and
-  // dB = T^T dY in units that fill the SMs its last wave of tiles leaves idle.
-  ProfScope p1(st, "split_t_pair", 1);
-  cudaError_t e = launch_split_pair(T_save, M, r, Tpair, st);
-  p1.done();
-  if (e != cudaSuccess) return cuda_fail(e);
+  // One launch: U = s dY B^T (and the bf16 pair of T) in the first units,
+  // the dX tiles, and dA = X^T U and dB = T^T dY in units that fill the SMs
+  // the last wave of tiles leaves idle.
   ProfScope p2(st, "fused_nf4_dx", 1);
-  e = launch_fused_dx(dY, codes, absmax_q, absmax_scale, Upair, A, M, K, N, r, dX, status, P, st, B, scale,
-                      reinterpret_cast<int*>(ws + wl.cd_off), X, Tpair, dA, dB);
+  const cudaError_t e = launch_fused_dx(dY, codes, absmax_q, absmax_scale, Upair, A, M, K, N, r, dX, status, P, st,
+                                        B, scale, reinterpret_cast<int*>(ws + wl.cd_off), X, T_save, Tpair, dA, dB);
   p2.done();
   if (e != cudaSuccess) return cuda_fail(e);
   return QLORA_OK;

@@ -80,6 +80,10 @@ struct PairArgs {
   int nmb;          // 64-row blocks of M (reduction depth of a tail unit)
   float* dA;        // [K x r]
   float* dB;        // [r x N]
+  // Input gradient: the rank units also write the bf16 pair of T (read by
+  // the dB tail units) from T as saved by the forward, for their rows.
+  const float* t_src;
+  uint16_t* t_pair;
   int nkb;          // main 64-deep stages
   int lora_kb;      // LoRA stages (hi and lo halves of the pair)
   int lora_mod;     // rp: LoRA stage lk reads the adapter at (64*lk) mod rp
@@ -282,11 +286,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           // 64 tokens per stage: this CTA's 2 x 128 result rows of the
           // activation (four 64-column boxes) and its rp columns of the pair.
           const bool is_da = tj < args.da_units;
-          if (i == 0 && is_da) {
+          if (i == 0) {
             bool ok = true;
             for (int m = 0; m < args.r_units && ok; ++m) ok = wait_count(args.ctr + 2 + m, 2, ctx);
             if (!ok) break;
-            fence_proxy_async_global();  // U is written by this launch's rank units
+            fence_proxy_async_global();  // the U and T pairs are written by this launch's rank units
           }
           const CUtensorMap* am = is_da ? &tm.a_da : &tm.a_db;
           const CUtensorMap* bm = is_da ? &tm.b_da : &tm.b_db;
@@ -425,7 +429,40 @@ __global__ void __launch_bounds__(kThreads, 1)
       asm volatile("bar.sync 1, 256;" ::: "memory");
       const int64_t blocks_per_row = args.w_cols / 64;
       if (runit || tunit) {
-        // rank and tail units read no weight
+        // Rank and tail units read no weight.  In the input gradient the
+        // rank units' idle decoder threads write the bf16 pair of the saved
+        // T for the unit's rows (one row per thread), for the dB tail units.
+        if (runit && args.t_pair) {
+          const int local = threadIdx.x - 128;  // 0..255
+          const int64_t row = static_cast<int64_t>(tile_m) * kPairRows + (local >> 7) * 256 + rank * 128 + (local & 127);
+          const int rp = args.lora_mod;
+          if (row < args.rows) {
+            const float* ts = args.t_src + row * args.r;
+            uint16_t* tp = args.t_pair + row * 2 * rp;
+#pragma unroll 1
+            for (int c0 = 0; c0 < rp; c0 += 8) {
+              float tv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+              if (c0 < args.r) {
+                const float4 t0 = __ldg(reinterpret_cast<const float4*>(ts + c0));
+                const float4 t1 = __ldg(reinterpret_cast<const float4*>(ts + c0 + 4));
+                tv[0] = t0.x; tv[1] = t0.y; tv[2] = t0.z; tv[3] = t0.w;
+                tv[4] = t1.x; tv[5] = t1.y; tv[6] = t1.z; tv[7] = t1.w;
+              }
+              uint32_t hi[4], lo[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const __nv_bfloat16 h0 = __float2bfloat16_rn(tv[2 * e]);
+                const __nv_bfloat16 h1 = __float2bfloat16_rn(tv[2 * e + 1]);
+                const __nv_bfloat16 l0 = __float2bfloat16_rn(__fsub_rn(tv[2 * e], __bfloat162float(h0)));
+                const __nv_bfloat16 l1 = __float2bfloat16_rn(__fsub_rn(tv[2 * e + 1], __bfloat162float(h1)));
+                hi[e] = __bfloat16_as_ushort(h0) | (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
+                lo[e] = __bfloat16_as_ushort(l0) | (static_cast<uint32_t>(__bfloat16_as_ushort(l1)) << 16);
+              }
+              *reinterpret_cast<uint4*>(tp + c0) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+              *reinterpret_cast<uint4*>(tp + rp + c0) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            }
+          }
+        }
       } else if (!MNB) {
         // Thread d decodes weight row n (this CTA's half), one block per stage.
         const int64_t n = static_cast<int64_t>(tile_n) * kPairCols + rank * 128 + d;
@@ -770,8 +807,8 @@ cudaError_t launch_fused_fwd(const uint16_t* X, const uint8_t* codes, const uint
 cudaError_t launch_fused_dx(const uint16_t* dY, const uint8_t* codes, const uint8_t* absmax_q,
                             const float* absmax_scale, uint16_t* Upair, const uint16_t* A, int64_t M, int64_t K,
                             int64_t N, int r, uint16_t* dX, int* status, const Nf4Params& P, cudaStream_t stream,
-                            const uint16_t* B, float scale, int* ctr, const uint16_t* X, const uint16_t* Tpair,
-                            float* dA, float* dB) {
+                            const uint16_t* B, float scale, int* ctr, const uint16_t* X, const float* T_save,
+                            uint16_t* Tpair, float* dA, float* dB) {
   const int rp = lora_pad(r);
   CUtensorMap mD, mC, mU, mA, mR;
   if (!make_map_2d(&mD, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dY, N, M, N * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -797,7 +834,7 @@ cudaError_t launch_fused_dx(const uint16_t* dY, const uint8_t* codes, const uint
   if (ctr && dA && dB) {
     // dA = X^T U and dB^T = dY^T T: 64 tokens x 64 result rows per box
     const int64_t ps = static_cast<int64_t>(rp) * 4;
-    if (!X || !Tpair ||
+    if (!X || !T_save || !Tpair ||
         !make_map_2d(&tails.a_da, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, K * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map_2d(&tails.b_da, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Upair, 2 * rp, M, ps, 64, 64,
                      CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -813,6 +850,8 @@ cudaError_t launch_fused_dx(const uint16_t* dY, const uint8_t* codes, const uint
     args.nmb = static_cast<int>((M + 63) / 64);
     args.dA = dA;
     args.dB = dB;
+    args.t_src = T_save;
+    args.t_pair = Tpair;
   }
   args.nkb = static_cast<int>((N + 63) / 64);
   args.lora_kb = 2 * rp / 64;

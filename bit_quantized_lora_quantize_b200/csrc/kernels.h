@@ -46,15 +46,15 @@ cudaError_t launch_fused_fwd(const uint16_t* X, const uint8_t* codes, const uint
 
 // Fused dequant-GEMM, input gradient: dX[M,K] = dY[M,N] W'[N,K] + (U_hi + U_lo)[M,r] A[K,r]^T.
 // With `ctr` the kernel also computes U = s dY B^T (its pair in Upair) the
-// same way, and, when dA and dB are given, dA = X^T U and dB = T^T dY
-// (Tpair: the bf16 pair of T, written before this launch); with
+// same way, and, when dA and dB are given, dA = X^T U and dB = T^T dY (the
+// rank units write the bf16 pair of T_save into Tpair for that); with
 // ctr == nullptr Upair comes from the previous kernel.
 cudaError_t launch_fused_dx(const uint16_t* dY, const uint8_t* codes, const uint8_t* absmax_q,
                             const float* absmax_scale, uint16_t* Upair, const uint16_t* A, int64_t M, int64_t K,
                             int64_t N, int r, uint16_t* dX, int* status, const Nf4Params& P, cudaStream_t stream,
                             const uint16_t* B = nullptr, float scale = 0.0f, int* ctr = nullptr,
-                            const uint16_t* X = nullptr, const uint16_t* Tpair = nullptr, float* dA = nullptr,
-                            float* dB = nullptr);
+                            const uint16_t* X = nullptr, const float* T_save = nullptr, uint16_t* Tpair = nullptr,
+                            float* dA = nullptr, float* dB = nullptr);
 
 // Counter ints one fused launch with rank units needs for M rows.
 int fused_ctr_ints(int64_t M);
@@ -69,38 +69,5 @@ cudaError_t launch_small_m_fwd(const uint16_t* X, const uint8_t* codes, const ui
                                const float* absmax_scale, const uint16_t* A, const uint16_t* B, int64_t M,
                                int64_t K, int64_t N, int r, float scale, uint16_t* Y, float* T_save, uint16_t* Tpair,
                                void* scratch, int* status, const Nf4Params& P, cudaStream_t stream);
-
-// Rank-r products (reduction split over the CTAs of a cluster, partial tiles
-// summed in rank order through distributed shared memory):
-//   kXA   T  = s * X A          [M, r]   -> f32 (may be null) and pair
-//   kDyBt U  = s * dY B^T       [M, r]   -> f32 (may be null) and pair
-//   kTtDy dB = T^T dY  (fp32)   [r, N]   P1 = T pair
-//   kXtU  dA = X^T U   (fp32)   [K, r]   P1 = U pair
-enum class SkinnyKind { kXA, kDyBt, kTtDy, kXtU };
-
-struct SkinnyPlan {
-  int tiles;   // 128-row output tiles
-  int nkb;     // 64-deep reduction blocks
-  int kps;     // blocks per split
-  int splits;  // CTAs (one cluster) per tile
-  int bn;      // accumulator columns (rp for T and U, 2rp for dA, dB)
-};
-
-struct SkinnyOut {
-  float* f32;
-  uint16_t* pair;
-};
-
-SkinnyPlan plan_skinny(SkinnyKind kind, int64_t M, int64_t K, int64_t N, int r);
-
-// `scratch` (16-byte aligned, skinny_scratch_bytes of this product) holds the
-// splits' partial tiles in global memory; null keeps them in shared memory and
-// sums them through distributed shared memory instead.
-size_t skinny_scratch_bytes(SkinnyKind kind, int64_t M, int64_t K, int64_t N, int r);
-cudaError_t launch_skinny(SkinnyKind kind, const uint16_t* P0, const uint16_t* P1, int64_t M, int64_t K, int64_t N,
-                          int r, float scale, SkinnyOut out, float* scratch, int* status, cudaStream_t stream);
-
-// Pair matrix of a float32 [rows x r] matrix.
-cudaError_t launch_split_pair(const float* v, int64_t rows, int r, uint16_t* pair, cudaStream_t stream);
 
 }  // namespace qlora

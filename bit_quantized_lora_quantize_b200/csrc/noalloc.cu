@@ -16,7 +16,8 @@
 // with cudaGetSymbolAddress and keeps it; that first call should therefore
 // come before any stream capture on that device.  All calls on a device share
 // the array and it keeps the previous call's contents: each call clears the
-// status word it needs at zero and overwrites everything else it reads, and
+// status word and counters it needs at zero and overwrites everything else it
+// reads, and
 // calls that overlap on the GPU (different streams, or different host threads
 // without ordering) race on it.
 #include <cstdint>
@@ -80,23 +81,26 @@ extern "C" qlora_status qlora_linear_fwd_noalloc(const uint16_t* X, int64_t M, i
                         reinterpret_cast<uintptr_t>(Y) | reinterpret_cast<uintptr_t>(T_save);
   if ((mis & 15u) || (reinterpret_cast<uintptr_t>(absmax_scale) & 3u)) return QLORA_ERR_ALIGNMENT;
 
-  // Scratch layout: [status word][T pair: bf16 M x 2rp].
+  // Scratch layout: [status word][counters of the GEMM launch][T pair: bf16 M x 2rp].
+  const size_t ctr_bytes = round_up256(static_cast<size_t>(fused_ctr_ints(M)) * 4);
   const size_t pair_bytes = round_up256(static_cast<size_t>(M) * 2 * lora_pad(r) * 2);
-  if (kStatusBytes + pair_bytes > kNoAllocScratchBytes) return QLORA_ERR_WORKSPACE;
+  if (kStatusBytes + ctr_bytes + pair_bytes > kNoAllocScratchBytes) return QLORA_ERR_WORKSPACE;
 
   void* base = nullptr;
   cudaError_t e = scratch_address(&base);
   if (e != cudaSuccess) return QLORA_ERR_CUDA;
   unsigned char* ws = static_cast<unsigned char*>(base);
   int* status = reinterpret_cast<int*>(ws);
-  uint16_t* Tpair = reinterpret_cast<uint16_t*>(ws + kStatusBytes);
+  int* ctr = reinterpret_cast<int*>(ws + kStatusBytes);
+  uint16_t* Tpair = reinterpret_cast<uint16_t*>(ws + kStatusBytes + ctr_bytes);
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
 
-  // Clear the status word: a call that timed out earlier may have left it set.
-  e = cudaMemsetAsync(ws, 0, sizeof(int), st);
+  // Clear the status word and the counters: a call that timed out earlier
+  // may have left them set.  Then the one GEMM launch (T = s X A in its first
+  // units, then the output tiles).
+  e = cudaMemsetAsync(ws, 0, kStatusBytes + ctr_bytes, st);
   if (e == cudaSuccess)
-    e = launch_skinny(SkinnyKind::kXA, X, A, M, K, N, r, scale, SkinnyOut{T_save, Tpair}, nullptr, status, st);
-  if (e == cudaSuccess)
-    e = launch_fused_fwd(X, codes, absmax_q, absmax_scale, Tpair, B, M, K, N, r, Y, status, nf4_params(), st);
+    e = launch_fused_fwd(X, codes, absmax_q, absmax_scale, Tpair, B, M, K, N, r, Y, status, nf4_params(), st, A,
+                         T_save, scale, ctr);
   return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }

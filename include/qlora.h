@@ -123,11 +123,13 @@ QLORA_API qlora_status qlora_dequantize_nf4(const uint8_t* codes, const uint8_t*
  *                 zeros again before the next call.
  * Supported: K % 64 == 0, N % 8 == 0, r % 8 == 0 with 8 <= r <= 128,
  * M, N, K < 2^31.  Otherwise QLORA_ERR_UNSUPPORTED.
- * For M <= 128 the whole forward is one kernel whose thread blocks wait for
- * one another (cooperative launch: all of them must be resident at once);
- * if the device cannot hold them next to other work the call returns
- * QLORA_ERR_CUDA and launches nothing.  Sums are taken in a fixed order:
- * results are bit-reproducible run to run.
+ * The forward is one kernel launch.  For M <= 128 its thread blocks wait
+ * for one another (cooperative launch: all of them must be resident at
+ * once); if the device cannot hold them next to other work the call returns
+ * QLORA_ERR_CUDA and launches nothing.  For larger M, blocks that finished
+ * T for a 512-row block release the output tiles of those rows (work is
+ * handed out in that order, so no residency is needed).  Sums are taken in a
+ * fixed order: results are bit-reproducible run to run.
  */
 QLORA_API qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, int64_t K, int64_t N, const uint8_t* codes,
                               const uint8_t* absmax_q, const float* absmax_scale, const uint16_t* A,
@@ -169,18 +171,22 @@ QLORA_API qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, c
  *   The call allocates nothing:
  *   its scratch is one fixed 16 MiB device array inside this library, which
  *   every GPU that loads the library keeps until the process exits.
- *   - Shapes whose forward scratch (status word + bf16 pair of T, i.e.
- *     256 + 4*M*rp bytes with rp = r rounded up to 64) exceeds 16 MiB return
- *     QLORA_ERR_WORKSPACE and launch nothing; 4096 tokens at r = 64 need
- *     1 MiB, so up to 32768 tokens fit at r <= 64.
+ *   - Shapes whose forward scratch (status word, counters and the bf16 pair
+ *     of T: 256 + round256(4*(2 + ceil(M/512))) + round256(4*M*rp) bytes with
+ *     rp = r rounded up to 64) exceeds 16 MiB return QLORA_ERR_WORKSPACE and
+ *     launch nothing; 4096 tokens at r = 64 need about 1 MiB, so up to 32768
+ *     tokens fit at r <= 64.
  *   - The first call on a device (with that device current, and `stream`
  *     belonging to it) looks up the array's device address once; make that
  *     first call before any stream capture on that device.
  *   - All calls on a device share the array.  Calls that may overlap on the
  *     GPU (other streams, or host threads without ordering) race and must be
  *     serialised by the caller.
- *   - Each call clears the status word it uses; a pipeline timeout inside
- *     this call is not reported (qlora_check_status needs a workspace).
+ *   - Each call clears the status word and counters it uses; a pipeline
+ *     timeout inside this call is not reported (qlora_check_status needs a
+ *     workspace).
+ *   - For M > 128 it runs the same GEMM launch as qlora_linear_fwd and gives
+ *     the same bits.
  */
 QLORA_API qlora_status qlora_linear_fwd_noalloc(const uint16_t* X, int64_t M, int64_t K, int64_t N,
                                                 const uint8_t* codes, const uint8_t* absmax_q,
