@@ -129,7 +129,9 @@ __device__ __forceinline__ Nf4Thresholds make_thresholds(const Nf4Params& P, flo
   return T;
 }
 
-// Codes of two bf16 values (low half, high half) -> code in bits 0-3 and 16-19.
+// Codes of two bf16 values (low half, high half): the low byte of each
+// 16-bit half holds that value's code in both nibbles (bits 8-15 are not
+// defined).  A 4-step binary search over the 15 thresholds.
 __device__ __forceinline__ uint32_t encode_pair(const Nf4Thresholds& T, uint32_t x) {
   const uint32_t m3 = set_ge_bf16x2(x, T.t[7]);
   const uint32_t m2 = set_ge_bf16x2(x, lop3_sel(T.t[3], T.t[11], m3));
@@ -143,19 +145,20 @@ __device__ __forceinline__ uint32_t encode_pair(const Nf4Thresholds& T, uint32_t
   const uint32_t e0 = lop3_sel(d0, d1, m2);
   const uint32_t e1 = lop3_sel(d2, d3, m2);
   const uint32_t m0 = set_ge_bf16x2(x, lop3_sel(e0, e1, m3));
-  const uint32_t r1 = lop3_sel(m2, m3, 0x00080008u);  // bit 3 from m3, rest from m2
-  const uint32_t r2 = lop3_sel(m0, m1, 0x00020002u);  // bit 1 from m1, rest from m0
-  return lop3_sel(r2, r1, 0x000C000Cu) & 0x000F000Fu;
+  const uint32_t r1 = lop3_sel(m2, m3, 0x00880088u);  // bits 3 and 7 from m3, 2 and 6 from m2
+  const uint32_t r2 = lop3_sel(m0, m1, 0x00220022u);  // bits 1 and 5 from m1, 0 and 4 from m0
+  return lop3_sel(r2, r1, 0x00CC00CCu);
 }
 
-// Four pairs (8 elements in order) -> one packed 32-bit code word.
-__device__ __forceinline__ uint32_t pack_codes8(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3) {
-  // c_i: code of element 2i at bits 0-3, element 2i+1 at bits 16-19.
-  const uint32_t v01 = c0 | (c1 << 8);
-  const uint32_t v23 = c2 | (c3 << 8);
-  const uint32_t b01 = (v01 << 4) | (v01 >> 16);  // bytes 0,1 = e0e1, e2e3
-  const uint32_t b23 = (v23 << 4) | (v23 >> 16);
-  return prmt(b01, b23, 0x5410);
+// Four encoded pairs (8 elements in order) -> one packed 32-bit code word,
+// byte b = code of element 2b in the high nibble, element 2b + 1 in the low.
+__device__ __forceinline__ uint32_t pack_codes8(uint32_t d0, uint32_t d1, uint32_t d2, uint32_t d3) {
+  // bytes [e0 e0, e1 e1, e2 e2, e3 e3], then byte 0 = e0 | e1, byte 2 = e2 | e3
+  const uint32_t wa = prmt(d0, d1, 0x6420u);
+  const uint32_t wb = prmt(d2, d3, 0x6420u);
+  const uint32_t ya = lop3_sel(wa >> 8, wa, 0xF0F0F0F0u);
+  const uint32_t yb = lop3_sel(wb >> 8, wb, 0xF0F0F0F0u);
+  return prmt(ya, yb, 0x6420u);
 }
 
 }  // namespace qlora

@@ -40,7 +40,20 @@ __device__ __forceinline__ uint32_t chunk_pos(int row, int j) { return row * 128
 // holding a partial last block (numel % 64 != 0) is staged with plain loads
 // in the same layout.
 constexpr int kQuantStages = 2;
-constexpr int kQuantSmem = kQuantStages * kGroupElems * 2 + 1024 + 256 * 4 + 128;
+// Stages | thresholds per bf16 mantissa (128 rows x 16 bf16) | fp32(k/255)
+// as double (256) | barriers, warp maxima, abort flag.
+constexpr int kThrOff = kQuantStages * kGroupElems * 2;
+constexpr int kLvlOff = kThrOff + 128 * 16 * 2;
+constexpr int kQuantSmem = kLvlOff + 256 * 8 + 128 + 1024;
+
+// The thresholds T_j = RU_bf16(B_j * c) of a block constant c = m * 2^e
+// (m in [1, 2), 128 bf16 mantissas) are RU_bf16(B_j * m) * 2^e: rounding up
+// to a binary grid commutes with scaling by a power of two while every value
+// stays normal.  With the biased exponent of c in [kFastExpLo, 254] every
+// |T_j| (at least 2^-5 * 2^(e - 127) for the smallest boundary) is normal, so
+// the threshold is the table entry of m with e - 127 added to its exponent
+// field; other constants (subnormal or non-finite) take the exact product.
+constexpr int kFastExpLo = 6;
 
 __global__ void __launch_bounds__(kThreads, 3)
     quantize_nf4_kernel(const __grid_constant__ CUtensorMap tmW, const uint16_t* __restrict__ W, int64_t numel,
@@ -49,7 +62,8 @@ __global__ void __launch_bounds__(kThreads, 3)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* buf = smem;                                                   // 2 x 32 KB
-  float* lvl2 = reinterpret_cast<float*>(smem + kQuantStages * kGroupElems * 2);  // fp32(k/255)
+  uint16_t* thr = reinterpret_cast<uint16_t*>(smem + kThrOff);           // [128][16] bf16
+  double* lvl2 = reinterpret_cast<double*>(smem + kLvlOff);              // fp32(k/255), exact
   uint64_t* bar = reinterpret_cast<uint64_t*>(lvl2 + 256);
   float* warp_max = reinterpret_cast<float*>(bar + kQuantStages);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(warp_max + kThreads / 32);
@@ -61,7 +75,12 @@ __global__ void __launch_bounds__(kThreads, 3)
   const int64_t nbytes = (numel + 1) / 2;
   const bool ragged_tail = (numel % kBlock) != 0;  // last group staged with plain loads
 
-  lvl2[tid] = level2_value(tid);
+  lvl2[tid] = static_cast<double>(level2_value(tid));
+  for (int i = tid; i < 128 * 16; i += kThreads) {
+    const int m = i >> 4, j = i & 15;
+    const float cm = __uint_as_float(0x3F800000u | (static_cast<uint32_t>(m) << 16));  // 1 + m/128
+    thr[i] = j < 15 ? static_cast<uint16_t>(threshold_pair(P.bnd[j], cm)) : static_cast<uint16_t>(0);
+  }
   if (tid == 0) {
     for (int s = 0; s < kQuantStages; ++s) mbar_init(&bar[s], 1);
     *abort_flag = 0;
@@ -152,9 +171,10 @@ __global__ void __launch_bounds__(kThreads, 3)
         int k0 = __float2int_rn(n2 * 255.0f);
         k0 = max(2, min(253, k0));
         double best = 4.0;
+        const double n2d = static_cast<double>(n2);
 #pragma unroll
         for (int d = -2; d <= 2; ++d) {
-          const double dist = fabs(static_cast<double>(n2) - static_cast<double>(lvl2[k0 + d]));
+          const double dist = fabs(n2d - lvl2[k0 + d]);
           if (dist < best) {
             best = dist;
             code2 = static_cast<uint32_t>(k0 + d);
@@ -166,7 +186,22 @@ __global__ void __launch_bounds__(kThreads, 3)
     if (tid == 0) absmax_scale[g] = c1;
 
     // 4-bit codes of the block.
-    const Nf4Thresholds T = make_thresholds(P, c);
+    Nf4Thresholds T;
+    {
+      const uint32_t cb = __float_as_uint(c > 0.0f ? c : 1.0f);  // all-zero block: every code is 7
+      const uint32_t e = cb >> 23;                                // c > 0: no sign bit
+      if (e >= kFastExpLo && e <= 254) {
+        const uint4* row = reinterpret_cast<const uint4*>(thr + ((cb >> 16) & 0x7Fu) * 16);
+        const uint4 r0 = row[0], r1 = row[1];
+        const uint32_t w[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+        // e - 127 added to the exponent field of both halves
+        const uint32_t de = (e - 127u) * 0x00800080u;
+#pragma unroll
+        for (int j = 0; j < 15; ++j) T.t[j] = prmt(w[j >> 1], 0, (j & 1) ? 0x3232u : 0x1010u) + de;
+      } else {
+        T = make_thresholds(P, c);
+      }
+    }
     uint32_t out[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j)

@@ -60,6 +60,26 @@ def test_every_bf16_pattern():
         assert_codec_equal(synthetic.to_bf16(blocks.reshape(-1)))
 
 
+def test_every_block_constant_mantissa():
+    """Thresholds of a block constant c = m * 2^e come from a per-mantissa
+    table scaled by 2^e: every one of the 128 bf16 mantissas, at three
+    exponents and next to the smallest exponent that uses the table, with
+    every bf16 value of [-c, c] above c * 2^-10 spread over blocks whose
+    first element is c (so c is each block's absmax)."""
+    bits = (np.arange(65536, dtype=np.uint32) << 16).view(np.float32)
+    base = bits[np.isfinite(bits) & (np.abs(bits) >= 2.0 ** -10) & (np.abs(bits) < 2.0)]
+    blocks = []
+    for scale in (1.0, 2.0 ** -100, 2.0 ** 100, 2.0 ** -121, 2.0 ** -122):
+        for m in range(128):
+            c = np.float32((1.0 + m / 128.0) * scale)
+            xs = base[np.abs(base) <= 1.0 + m / 128.0].astype(np.float64) * scale
+            xs = np.concatenate([xs, np.zeros((-len(xs)) % 63)]).astype(np.float32).reshape(-1, 63)
+            blocks.append(np.concatenate([np.full((len(xs), 1), c, np.float32), xs], axis=1))
+            if scale in (2.0 ** -121, 2.0 ** -122) and m >= 3:
+                break
+    assert_codec_equal(synthetic.to_bf16(np.concatenate(blocks).reshape(-1)))
+
+
 def test_dequantize_arbitrary_packed_input():
     rng = np.random.default_rng(4)
     n = 64 * 256 * 3 + 64 * 7
