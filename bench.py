@@ -270,8 +270,6 @@ def small_m_sweep(q, synthetic, dev, flush, iters=10):
                     k_us = ms * 1e3 / max(calls, 1)
                     ent.update({"kernel": name, "kernel_us": k_us,
                                 "kernel_frac_hbm": nf4_bytes / (k_us * 1e-6) / 1e9 / peaks["hbm_gbs"]})
-                elif name == "lora_down_xa":
-                    ent["lora_down_us"] = ms * 1e3 / max(calls, 1)
             out.append(ent)
     return out
 
