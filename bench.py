@@ -349,6 +349,9 @@ def run_ours(args, rank, world, local_rank):
     fl_step = flops_fwd(M, K, N, r) + flops_bwd(M, K, N, r)
     value = fl_step * world / (ms_per_step * 1e-3) / 1e12
     tokens_per_s = M * world / (ms_per_step * 1e-3)
+    # The same step time with only the dense products counted (4MNK: the
+    # frozen-weight GEMMs of forward and input gradient).
+    value_dense = 4 * M * N * K * world / (ms_per_step * 1e-3) / 1e12
 
     # ---------------- end to end through the public API with host buffers
     pin = lambda t: t.cpu().pin_memory()  # noqa: E731
@@ -409,6 +412,7 @@ def run_ours(args, rank, world, local_rank):
         "config": dict(WORKLOAD, parallelism=f"dp{world}", global_batch_tokens=M * world,
                        l2="flushed between timed steps (256 MB write)"),
         "tokens_per_s": tokens_per_s,
+        "tflops_dense_only": value_dense,
         "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peaks["bf16_tflops"],
                      "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": traffic_for(dom),
                      "peak_source": f"{peaks['source']} bf16 burst", "ms_per_launch": dom_ms},
