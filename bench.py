@@ -202,10 +202,13 @@ def run_reference(args, rank, world):
     v = sorted(vals)[len(vals) // 2]
     cb = dict(samples[-1])
     cb["value"] = v
+    # The whole step's flops at the sample's rate: the time one full step would take.
+    M, K, N, r = WORKLOAD["M"], WORKLOAD["K"], WORKLOAD["N"], WORKLOAD["r"]
+    ms_full = (flops_fwd(M, K, N, r) + flops_bwd(M, K, N, r)) / (v * 1e12) * 1e3
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_full, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": dict(WORKLOAD), "cpu_baseline": cb,
+            "config": dict(WORKLOAD), "cpu_baseline": cb, "tokens_per_s": M / (ms_full * 1e-3),
             "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 

@@ -1,5 +1,8 @@
-"""Host-side logic of bench.py that needs no GPU: the clock sampler, run
-against a fake NVML module in the child process it starts."""
+"""Host-side logic of bench.py that needs no GPU: the clock sampler (run
+against a fake NVML module in the child process it starts), the rule that
+keeps a committed DRAM-traffic figure only while its kernel's sources are
+unchanged, and the oracle reference arm's JSON line."""
+import sys
 import time
 
 import pytest
@@ -51,3 +54,45 @@ def test_clock_sampler_without_nvml_returns_none(tmp_path, monkeypatch):
     c.start()
     assert c.poller is None
     assert c.stop() is None
+
+
+def test_traffic_entry_goes_null_when_the_kernel_source_changes(tmp_path, monkeypatch):
+    """The committed DRAM bytes of a kernel are reported only while the
+    hashed sources are the ones the ncu capture was taken of."""
+    import hashlib
+    import json
+
+    import bench
+
+    csrc = tmp_path / "bit_quantized_lora_quantize_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "k.cu").write_text("kernel v1")
+    (csrc / "h.cuh").write_text("header")
+    digest = hashlib.sha256(b"kernel v1" + b"header").hexdigest()[:16]
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(
+        {"gemm": {"sources": ["k.cu", "h.cuh"], "dram_bytes_per_launch": 123, "sources_sha256_16": digest}}))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.traffic_for("gemm") == 123
+    assert bench.traffic_for("other") is None
+    (csrc / "k.cu").write_text("kernel v2")
+    assert bench.traffic_for("gemm") is None
+
+
+def test_reference_arm_prints_the_contract_line():
+    """`bench.py --impl reference` times the oracle on the host cores and
+    prints one JSON line with the keys the driver reads."""
+    import json
+    import pathlib
+    import subprocess
+
+    root = pathlib.Path(__file__).resolve().parents[1]
+    out = subprocess.run([sys.executable, str(root / "bench.py"), "--impl", "reference", "--steps", "1",
+                          "--warmup", "0"], cwd=root, capture_output=True, text=True, timeout=600)
+    assert out.returncode == 0, out.stderr[-2000:]
+    d = json.loads(out.stdout.strip().splitlines()[-1])
+    assert d["impl"] == "reference" and d["unit"] == "TFLOP/s" and d["higher_is_better"] is True
+    assert d["value"] > 0 and d["ms_per_step"] > 0 and d["tokens_per_s"] > 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"] == {"value": d["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    assert d["config"]["workload"] == "llama7b_attn_proj_qlora_linear"
