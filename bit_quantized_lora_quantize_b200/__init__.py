@@ -13,6 +13,8 @@ from .qlora import (  # noqa: F401
     lib,
     new_workspace,
     qlora_check_status,
+    qlora_get_wait_timeout,
+    qlora_set_wait_timeout,
     qlora_dequantize_nf4,
     qlora_linear_bwd,
     qlora_linear_fwd,

@@ -1,6 +1,7 @@
 // C ABI of the library: argument validation, workspace layout and the
 // sequence of kernel launches for each call (declared in include/qlora.h).
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -13,6 +14,7 @@
 #include <cuda_runtime.h>
 
 #include "../../include/qlora.h"
+#include "abi_internal.h"
 #include "kernels.h"
 #include "nf4_host.h"
 #include "tensor_map.h"
@@ -23,12 +25,8 @@ namespace {
 
 thread_local std::string g_last_cuda_error;
 
-qlora_status cuda_fail(cudaError_t e) {
-  g_last_cuda_error = cudaGetErrorString(e);
-  return QLORA_ERR_CUDA;
-}
-
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+// Limit of every bounded wait in the kernels (qlora_set_wait_timeout).
+std::atomic<uint64_t> g_wait_ns{kWaitTimeoutNs};
 
 constexpr size_t kStatusBytes = 256;
 
@@ -52,13 +50,6 @@ WsLayout ws_layout(int64_t M, int64_t K, int64_t N, int r) {
   w.sm_off = w.u_off + pair_bytes;
   w.total = w.sm_off + (M <= kSmallMMax ? round_up(small_m_workspace_bytes(M, N, r), 256) : 0);
   return w;
-}
-
-qlora_status check_linear_shape(int64_t M, int64_t K, int64_t N, int32_t r) {
-  if (M <= 0 || K <= 0 || N <= 0 || r <= 0) return QLORA_ERR_INVALID_ARG;
-  if (M >= (int64_t(1) << 31) || K >= (int64_t(1) << 31) || N >= (int64_t(1) << 31)) return QLORA_ERR_UNSUPPORTED;
-  if (K % 64 != 0 || N % 8 != 0 || r % 8 != 0 || r > 128) return QLORA_ERR_UNSUPPORTED;
-  return QLORA_OK;
 }
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -102,31 +93,39 @@ cudaEvent_t prof_event() {
   return e;
 }
 
-struct ProfScope {
-  bool on;
-  cudaStream_t st;
-  const char* name;
-  int launches;
-  cudaEvent_t a = nullptr;
-  ProfScope(cudaStream_t s, const char* n, int l) : on(false), st(s), name(n), launches(l) {
-    std::lock_guard<std::mutex> g(g_prof_mu);
-    on = g_prof_on;
-    if (on) {
-      a = prof_event();
-      cudaEventRecord(a, st);
-    }
-  }
-  void done() {
-    if (!on) return;
-    std::lock_guard<std::mutex> g(g_prof_mu);
-    cudaEvent_t b = prof_event();
-    cudaEventRecord(b, st);
-    g_prof_recs.push_back({name, launches, a, b});
-    on = false;
-  }
-};
-
 }  // namespace
+
+qlora_status cuda_fail(cudaError_t e) {
+  g_last_cuda_error = cudaGetErrorString(e);
+  return QLORA_ERR_CUDA;
+}
+
+qlora_status check_linear_shape(int64_t M, int64_t K, int64_t N, int32_t r) {
+  if (M <= 0 || K <= 0 || N <= 0 || r <= 0) return QLORA_ERR_INVALID_ARG;
+  if (M >= (int64_t(1) << 31) || K >= (int64_t(1) << 31) || N >= (int64_t(1) << 31)) return QLORA_ERR_UNSUPPORTED;
+  if (K % 64 != 0 || N % 8 != 0 || r % 8 != 0 || r > 128) return QLORA_ERR_UNSUPPORTED;
+  return QLORA_OK;
+}
+
+uint64_t wait_limit_ns() { return g_wait_ns.load(std::memory_order_relaxed); }
+
+ProfScope::ProfScope(cudaStream_t s, const char* n, int l) : on(false), st(s), name(n), launches(l) {
+  std::lock_guard<std::mutex> g(g_prof_mu);
+  on = g_prof_on;
+  if (on) {
+    a = prof_event();
+    cudaEventRecord(a, st);
+  }
+}
+
+void ProfScope::done() {
+  if (!on) return;
+  std::lock_guard<std::mutex> g(g_prof_mu);
+  cudaEvent_t b = prof_event();
+  cudaEventRecord(b, st);
+  g_prof_recs.push_back({name, launches, a, b});
+  on = false;
+}
 
 bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, int64_t inner, int64_t rows,
                  int64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle swizzle) {
@@ -251,18 +250,41 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float
 }
 
 qlora_status qlora_check_status(void* workspace, void* stream) {
-  if (!workspace) return QLORA_ERR_INVALID_ARG;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaStreamSynchronize(st);
   if (e != cudaSuccess) return cuda_fail(e);
+  bool timed_out = false;
+  if (workspace) {
+    int word = 0;
+    e = cudaMemcpyAsync(&word, workspace, sizeof(int), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (word != 0) {
+      timed_out = true;
+      e = cudaMemsetAsync(workspace, 0, sizeof(int), st);
+      if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+      if (e != cudaSuccess) return cuda_fail(e);
+    }
+  }
+  // The status words inside the library (quantization, allocation-free
+  // forward) on the current device.
   int word = 0;
-  e = cudaMemcpy(&word, workspace, sizeof(int), cudaMemcpyDeviceToHost);
+  e = codec_status_take(st, &word);
   if (e != cudaSuccess) return cuda_fail(e);
-  if (word == 0) return QLORA_OK;
-  e = cudaMemset(workspace, 0, sizeof(int));
+  timed_out |= word != 0;
+  e = noalloc_status_take(st, &word);
   if (e != cudaSuccess) return cuda_fail(e);
-  return QLORA_ERR_TIMEOUT;
+  timed_out |= word != 0;
+  return timed_out ? QLORA_ERR_TIMEOUT : QLORA_OK;
 }
+
+qlora_status qlora_set_wait_timeout(uint64_t timeout_ns) {
+  if (timeout_ns > kMaxWaitTimeoutNs) return QLORA_ERR_INVALID_ARG;
+  g_wait_ns.store(timeout_ns == 0 ? kWaitTimeoutNs : timeout_ns, std::memory_order_relaxed);
+  return QLORA_OK;
+}
+
+uint64_t qlora_get_wait_timeout(void) { return wait_limit_ns(); }
 
 void qlora_nf4_codebook(float out[16]) {
   if (!out) return;

@@ -95,6 +95,7 @@ struct PairArgs {
   int64_t w_rows, w_cols;  // N, K of the packed weight
   int abs_tma;             // dX: 8-bit constant codes by TMA
   int* status;
+  uint64_t wait_ns;         // limit of every bounded wait
   Nf4Params nf4;
 };
 
@@ -116,8 +117,8 @@ struct PairSmem {
   static constexpr int offAbs = offC + kStages * kC;
   static constexpr int offLvl2 = offAbs + kStages * kAbs;
   static constexpr int offBar = offLvl2 + 1024;
-  // full, cfull, empty, decoded per stage; acc_full
-  static constexpr int kNumBars = 4 * kStages + 1;
+  // full, cfull, empty, decoded per stage; acc_full; one MMA drain per issuer
+  static constexpr int kNumBars = 4 * kStages + 3;
   static constexpr int offSlot = offBar + kNumBars * 8;
   static constexpr int offAbort = offSlot + 4;
   static constexpr int offUnit = offAbort + 4;
@@ -205,6 +206,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* empty = cfull + kStages;                               // local: MMA done with the stage
   uint64_t* decoded = empty + kStages;                             // leader: both CTAs' decoders
   uint64_t* acc_full = decoded + kStages;                          // local: accumulators ready
+  uint64_t* mma_drain = acc_full + 1;                              // leader: an issuer's MMAs ended (abort)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::offSlot);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::offAbort);
   int* unit_slot = reinterpret_cast<int*>(smem + L::offUnit);
@@ -221,6 +223,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&decoded[s], 2 * kDecWarps);
     }
     mbar_init(acc_full, 2);
+    mbar_init(&mma_drain[0], 1);
+    mbar_init(&mma_drain[1], 1);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -272,7 +276,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      const WaitCtx ctx{abort_flag, args.status, 21};
+      const WaitCtx ctx{abort_flag, args.status, 21, args.wait_ns};
       int issued = 0;
       for (int i = 0; i < total; ++i) {
         const int s = i % kStages;
@@ -362,14 +366,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++issued;
       }
       if (*abort_flag) {
+        // Let every copy this CTA pair issued land before the CTAs exit (the
+        // leader's full barrier counts both CTAs' activation bytes).
         for (int i = (issued > kStages ? issued - kStages : 0); i < issued; ++i) {
-          const uint64_t t0 = globaltimer_ns();
           const int s = i % kStages;
           const uint32_t ph = (i / kStages) & 1;
           const bool codes = i < args.nkb && !runit && !tunit;  // only these stages load codes
-          while (globaltimer_ns() - t0 < kWaitTimeoutNs &&
-                 !((!codes || mbar_try_wait(&cfull[s], ph)) && (rank != 0 || mbar_try_wait(&full[s], ph)))) {
-          }
+          if (codes) mbar_drain(&cfull[s], ph);
+          if (rank == 0) mbar_drain(&full[s], ph);
         }
       }
     }
@@ -381,7 +385,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // second; each commits to the stage and accumulator barriers (count 2).
     if (lane == 0 && rank == 0) {
       const int h = warp - 1;
-      const WaitCtx ctx{abort_flag, args.status, 22};
+      const WaitCtx ctx{abort_flag, args.status, 22, args.wait_ns};
       // M = 256 across the pair, N = 256 (each CTA supplies 128 columns of B).
       const uint32_t idesc_main = idesc_bf16_f32(256, 256, false, MNB);
       const uint32_t idesc_lora = idesc_bf16_f32(256, 256, false, !MNB);
@@ -415,14 +419,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         umma_commit_pair(&empty[s]);
       }
-      if (ok) umma_commit_pair(acc_full);
+      if (ok) {
+        umma_commit_pair(acc_full);
+      } else {
+        // Aborted: wait until the MMAs this thread issued have ended, so that
+        // neither CTA frees its TMEM or leaves while they still read the
+        // pair's shared memory.
+        umma_commit_pair(&mma_drain[h]);
+        mbar_drain(&mma_drain[h], 0);
+      }
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ decoders (warps 4-11)
     // Two groups of four warps take alternate stages; in each group thread d
     // decodes one 64-weight block of this CTA's half of the weight tile.
     {
-      const WaitCtx ctx{abort_flag, args.status, 23};
+      const WaitCtx ctx{abort_flag, args.status, 23, args.wait_ns};
       const int grp = (warp - 4) >> 2;          // 0: even stages, 1: odd stages
       const int d = (threadIdx.x - 128) & 127;  // 0..127
       lvl2[threadIdx.x - 128] = level2_value(threadIdx.x - 128);
@@ -575,7 +587,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // ------------------------------------------------------------ epilogue (warps 4-11)
     {
-      const WaitCtx ctx{abort_flag, args.status, 24};
+      const WaitCtx ctx{abort_flag, args.status, 24, args.wait_ns};
       const int q = warp & 3;
       const int h = (warp - 4) >> 2;  // accumulator (first or second M = 256 MMA)
       const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(acc_full, 0, ctx));
@@ -799,6 +811,7 @@ cudaError_t launch_fused_fwd(const uint16_t* X, const uint8_t* codes, const uint
   args.w_cols = K;
   args.abs_tma = 0;
   args.status = status;
+  args.wait_ns = wait_limit_ns();
   args.nf4 = P;
   const TailMaps none{mB, mB, mB, mB};
   return launch_pair<false>(mX, mC, mT, mB, mB, mR, none, args, stream);
@@ -866,6 +879,7 @@ cudaError_t launch_fused_dx(const uint16_t* dY, const uint8_t* codes, const uint
   args.w_cols = K;
   args.abs_tma = abs_tma ? 1 : 0;
   args.status = status;
+  args.wait_ns = wait_limit_ns();
   args.nf4 = P;
   return launch_pair<true>(mD, mC, mU, mA, mAbs, mR, tails, args, stream);
 }

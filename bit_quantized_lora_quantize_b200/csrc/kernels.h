@@ -9,6 +9,18 @@
 
 namespace qlora {
 
+// Limit of every bounded wait in the kernels, as set by
+// qlora_set_wait_timeout (kWaitTimeoutNs by default, at most
+// kMaxWaitTimeoutNs).  Each launch copies it into its arguments.
+constexpr uint64_t kMaxWaitTimeoutNs = 60000000000ull;  // 60 s
+uint64_t wait_limit_ns();
+
+// Status words the library keeps on the device for calls without a
+// workspace: each reads the current device's word (after the stream's work),
+// clears it if it was set and returns it in *word.
+cudaError_t codec_status_take(cudaStream_t stream, int* word);
+cudaError_t noalloc_status_take(cudaStream_t stream, int* word);
+
 // Launch attribute that lets a kernel start before its predecessor in the
 // stream has ended (programmatic dependent launch).  Every kernel launched
 // with it calls griddep_wait before it reads anything its predecessor writes

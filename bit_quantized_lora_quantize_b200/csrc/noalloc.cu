@@ -16,16 +16,18 @@
 // with cudaGetSymbolAddress and keeps it; that first call should therefore
 // come before any stream capture on that device.  All calls on a device share
 // the array and it keeps the previous call's contents: each call clears the
-// status word and counters it needs at zero and overwrites everything else it
-// reads, and
+// counters it needs at zero and overwrites everything else it reads, and
 // calls that overlap on the GPU (different streams, or different host threads
-// without ordering) race on it.
+// without ordering) race on it.  The first 256 bytes hold the status word: a
+// pipeline wait that gave up sets it, and qlora_check_status reports and
+// clears it (calls leave it alone, so a timeout stays visible until then).
 #include <cstdint>
 #include <mutex>
 
 #include <cuda_runtime.h>
 
 #include "../../include/qlora.h"
+#include "abi_internal.h"
 #include "kernels.h"
 #include "nf4_host.h"
 
@@ -63,6 +65,26 @@ cudaError_t scratch_address(void** out) {
 
 }  // namespace
 
+cudaError_t noalloc_status_take(cudaStream_t stream, int* word) {
+  *word = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  void* base = nullptr;
+  {
+    std::lock_guard<std::mutex> g(g_setup_mu);
+    if (dev >= 0 && dev < kMaxDevices) base = g_scratch_ptr[dev];
+  }
+  if (!base) return cudaSuccess;  // no allocation-free call ran on this device
+  e = cudaMemcpyAsync(word, base, sizeof(int), cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  if (e == cudaSuccess && *word != 0) {
+    e = cudaMemsetAsync(base, 0, sizeof(int), stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  }
+  return e;
+}
+
 }  // namespace qlora
 
 using namespace qlora;
@@ -73,13 +95,11 @@ extern "C" qlora_status qlora_linear_fwd_noalloc(const uint16_t* X, int64_t M, i
                                                  int32_t r, float scale, uint16_t* Y, float* T_save, void* stream) {
   if (!X || !codes || !absmax_q || !absmax_scale || !A || !B || !Y || !T_save) return QLORA_ERR_INVALID_ARG;
   if (!(scale == scale) || scale - scale != 0.0f) return QLORA_ERR_INVALID_ARG;  // NaN or infinite
-  if (M <= 0 || K <= 0 || N <= 0 || r <= 0) return QLORA_ERR_INVALID_ARG;
-  if (M >= (int64_t(1) << 31) || K >= (int64_t(1) << 31) || N >= (int64_t(1) << 31)) return QLORA_ERR_UNSUPPORTED;
-  if (K % 64 != 0 || N % 8 != 0 || r % 8 != 0 || r > 128) return QLORA_ERR_UNSUPPORTED;
-  const uintptr_t mis = reinterpret_cast<uintptr_t>(X) | reinterpret_cast<uintptr_t>(codes) |
-                        reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(B) |
-                        reinterpret_cast<uintptr_t>(Y) | reinterpret_cast<uintptr_t>(T_save);
-  if ((mis & 15u) || (reinterpret_cast<uintptr_t>(absmax_scale) & 3u)) return QLORA_ERR_ALIGNMENT;
+  const qlora_status sh = check_linear_shape(M, K, N, r);
+  if (sh != QLORA_OK) return sh;
+  if (!aligned16(X) || !aligned16(codes) || !aligned16(A) || !aligned16(B) || !aligned16(Y) || !aligned16(T_save) ||
+      (reinterpret_cast<uintptr_t>(absmax_scale) & 3u))
+    return QLORA_ERR_ALIGNMENT;
 
   // Scratch layout: [status word][counters of the GEMM launch][T pair: bf16 M x 2rp].
   const size_t ctr_bytes = round_up256(static_cast<size_t>(fused_ctr_ints(M)) * 4);
@@ -88,19 +108,21 @@ extern "C" qlora_status qlora_linear_fwd_noalloc(const uint16_t* X, int64_t M, i
 
   void* base = nullptr;
   cudaError_t e = scratch_address(&base);
-  if (e != cudaSuccess) return QLORA_ERR_CUDA;
+  if (e != cudaSuccess) return cuda_fail(e);
   unsigned char* ws = static_cast<unsigned char*>(base);
   int* status = reinterpret_cast<int*>(ws);
   int* ctr = reinterpret_cast<int*>(ws + kStatusBytes);
   uint16_t* Tpair = reinterpret_cast<uint16_t*>(ws + kStatusBytes + ctr_bytes);
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
 
-  // Clear the status word and the counters: a call that timed out earlier
-  // may have left them set.  Then the one GEMM launch (T = s X A in its first
-  // units, then the output tiles).
-  e = cudaMemsetAsync(ws, 0, kStatusBytes + ctr_bytes, st);
-  if (e == cudaSuccess)
-    e = launch_fused_fwd(X, codes, absmax_q, absmax_scale, Tpair, B, M, K, N, r, Y, status, nf4_params(), st, A,
-                         T_save, scale, ctr);
-  return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+  // Clear the counters (a call that timed out earlier may have left them
+  // set), then the one GEMM launch: T = s X A in its first units, then the
+  // output tiles.  For every M this is the pair GEMM of the large-M forward.
+  e = cudaMemsetAsync(ctr, 0, ctr_bytes, st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  ProfScope p(st, "fused_nf4_fwd", 1);
+  e = launch_fused_fwd(X, codes, absmax_q, absmax_scale, Tpair, B, M, K, N, r, Y, status, nf4_params(), st, A,
+                       T_save, scale, ctr);
+  p.done();
+  return e == cudaSuccess ? QLORA_OK : cuda_fail(e);
 }

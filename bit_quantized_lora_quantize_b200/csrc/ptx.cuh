@@ -65,29 +65,59 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
 // Every wait in the kernels is bounded.  A wait that gives up sets the CTA's
 // abort flag (shared memory) and the device status word, and returns false;
 // all other waits of the CTA then fall through, so that every thread still
-// reaches the end of the kernel, frees its TMEM and exits.
-constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s
+// reaches the end of the kernel, frees its TMEM and exits.  The limit is a
+// kernel argument (set at run time on the host, 2 s by default).  After an
+// abort, a CTA waits for the work it already started (copies in flight, its
+// own MMAs) with the fixed kDrainTimeoutNs instead: that work ends within
+// microseconds on a working device, so 2 ms is ample, and leaving earlier
+// would let a copy land in memory the CTA no longer owns.  (A pair barrier
+// whose phase also needs the peer CTA's copies may never complete when the
+// peer aborted before issuing them; the drain then ends at the bound.)
+constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // default limit, 2 s
+constexpr uint64_t kDrainTimeoutNs = 2000000ull;    // 2 ms
+// Below this limit a wait polls without the suspend hint and reads the
+// timer after every try, so that short limits are honoured.
+constexpr uint64_t kShortWaitNs = 1000000ull;
 
 struct WaitCtx {
   volatile int* abort_flag;  // shared
   int* status;               // global, may be null
   int site;                  // identifies the wait that timed out
+  uint64_t limit_ns;         // give up after this long
 };
+
+__device__ __forceinline__ bool wait_gave_up(const WaitCtx& ctx) {
+  *ctx.abort_flag = 1;
+  if (ctx.status) atomicCAS(ctx.status, 0, 0x100 + ctx.site);
+  return false;
+}
 
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtx& ctx) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
+  if (ctx.limit_ns < kShortWaitNs) {
+    while (true) {
+      if (mbar_try_wait(bar, parity)) return true;
+      if (*ctx.abort_flag) return false;
+      if (globaltimer_ns() - t0 > ctx.limit_ns) return wait_gave_up(ctx);
+    }
+  }
   while (true) {
 #pragma unroll 1
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait_sleep(bar, parity, 20000)) return true;
     if (*ctx.abort_flag) return false;
-    if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
-      *ctx.abort_flag = 1;
-      if (ctx.status) atomicCAS(ctx.status, 0, 0x100 + ctx.site);
-      return false;
-    }
+    if (globaltimer_ns() - t0 > ctx.limit_ns) return wait_gave_up(ctx);
   }
+}
+
+// Wait for a phase this CTA's own async work will complete (copies or MMAs it
+// issued), ignoring the abort flag; bounded by kDrainTimeoutNs.
+__device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity))
+    if (globaltimer_ns() - t0 > kDrainTimeoutNs) return false;
+  return true;
 }
 
 // ---------------------------------------------------------------- flags in global memory
@@ -107,14 +137,10 @@ __device__ __forceinline__ bool wait_count(const int* p, int need, const WaitCtx
   if (ld_acquire(p) >= need) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
-    __nanosleep(128);
+    if (ctx.limit_ns >= kShortWaitNs) __nanosleep(128);
     if (ld_acquire(p) >= need) return true;
     if (*ctx.abort_flag) return false;
-    if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
-      *ctx.abort_flag = 1;
-      if (ctx.status) atomicCAS(ctx.status, 0, 0x100 + ctx.site);
-      return false;
-    }
+    if (globaltimer_ns() - t0 > ctx.limit_ns) return wait_gave_up(ctx);
   }
 }
 

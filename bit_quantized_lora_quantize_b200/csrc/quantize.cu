@@ -55,10 +55,15 @@ constexpr int kQuantSmem = kLvlOff + 256 * 8 + 128 + 1024;
 // field; other constants (subnormal or non-finite) take the exact product.
 constexpr int kFastExpLo = 6;
 
+// Status word of the codec kernels on this device: a quantization whose copy
+// wait gave up records it here (the call has no workspace), and
+// qlora_check_status reports and clears it.
+__device__ int g_codec_status;
+
 __global__ void __launch_bounds__(kThreads, 3)
     quantize_nf4_kernel(const __grid_constant__ CUtensorMap tmW, const uint16_t* __restrict__ W, int64_t numel,
                         uint8_t* __restrict__ codes, uint8_t* __restrict__ absmax_q,
-                        float* __restrict__ absmax_scale, Nf4Params P) {
+                        float* __restrict__ absmax_scale, Nf4Params P, uint64_t wait_ns) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* buf = smem;                                                   // 2 x 32 KB
@@ -68,7 +73,7 @@ __global__ void __launch_bounds__(kThreads, 3)
   float* warp_max = reinterpret_cast<float*>(bar + kQuantStages);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(warp_max + kThreads / 32);
   const int tid = threadIdx.x;
-  const WaitCtx ctx{abort_flag, nullptr, 5};
+  const WaitCtx ctx{abort_flag, &g_codec_status, 5, wait_ns};
 
   const int64_t groups = (numel + kGroupElems - 1) / kGroupElems;
   const int64_t nb = (numel + kBlock - 1) / kBlock;
@@ -107,13 +112,13 @@ __global__ void __launch_bounds__(kThreads, 3)
     const uint32_t phase = (it >> 1) & 1;
     const int64_t gn = g + gridDim.x;
     if (tid == 0 && gn < groups) issue(gn, stage ^ 1);
-    // Bounded wait: a copy that never lands ends the loop (the caller sees
-    // undefined codes) instead of hanging the device.
+    // Bounded wait: a copy that never lands ends the loop (the status word
+    // records it and the codes are undefined) instead of hanging the device.
+    // Both stages' copies in flight land before the CTA exits.
     if (!__syncthreads_and(mbar_wait(&bar[stage], phase, ctx))) {
-      if (tid == 0 && gn < groups) {
-        const uint64_t t0 = globaltimer_ns();
-        while (!mbar_try_wait(&bar[stage ^ 1], ((it + 1) >> 1) & 1) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
-        }
+      if (tid == 0) {
+        mbar_drain(&bar[stage], phase);
+        if (gn < groups) mbar_drain(&bar[stage ^ 1], ((it + 1) >> 1) & 1);
       }
       break;
     }
@@ -299,8 +304,20 @@ cudaError_t launch_quantize_nf4(const uint16_t* W, int64_t numel, uint8_t* codes
   if (e != cudaSuccess) return e;
   const int64_t grid = std::min<int64_t>(groups, static_cast<int64_t>(sm_count) * 3);
   quantize_nf4_kernel<<<static_cast<unsigned>(grid), kThreads, kQuantSmem, stream>>>(map, W, numel, codes, absmax_q,
-                                                                                      absmax_scale, P);
+                                                                                      absmax_scale, P, wait_limit_ns());
   return cudaGetLastError();
+}
+
+cudaError_t codec_status_take(cudaStream_t stream, int* word) {
+  *word = 0;
+  cudaError_t e = cudaMemcpyFromSymbolAsync(word, g_codec_status, sizeof(int), 0, cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  if (e == cudaSuccess && *word != 0) {
+    static const int zero = 0;
+    e = cudaMemcpyToSymbolAsync(g_codec_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  }
+  return e;
 }
 
 cudaError_t launch_dequantize_nf4(const uint8_t* codes, const uint8_t* absmax_q, const float* absmax_scale,

@@ -111,8 +111,9 @@ struct SmallLayout {
   // decoder-group counts.
   static constexpr int kASlots = MP == 16 ? 12 : (MP == 128 ? 4 : 8);
   static constexpr int kAccCols = 2 * kIssuers * MP;  // two buffers x kIssuers accumulators
-  // full/consumed per stage, lfull/lempty per LoRA slot, afull per A slot, accfull/accempty x2
-  static constexpr int kNumBars = 2 * kStages + 2 * kLoraSlots + kASlots + 4;
+  // full/consumed per stage, lfull/lempty per LoRA slot, afull per A slot, accfull/accempty x2,
+  // one MMA drain per issuer
+  static constexpr int kNumBars = 2 * kStages + 2 * kLoraSlots + kASlots + 4 + 4;
   static constexpr int offSlot = offBar + kNumBars * 8;
   static constexpr int offAbort = offSlot + 4;
   static constexpr int kTotal = offAbort + 4;
@@ -158,6 +159,7 @@ struct SmallMArgs {
   float* t_l1;     // ceil(nT / 8) slots
   float* partial;  // kMaxGrid + 2 * tiles slots: (c + t) weight range, kMaxGrid + tiles + t LoRA
   int* status;
+  uint64_t wait_ns;  // limit of every bounded wait
   Nf4Params nf4;
 };
 
@@ -177,11 +179,7 @@ __device__ __forceinline__ bool wait_t_ready(const SmallMArgs& a, const WaitCtx&
     __nanosleep(64);
     if (ld_acquire(a.t_ready) >= kReadyCount) return true;
     if (*ctx.abort_flag) return false;
-    if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
-      *ctx.abort_flag = 1;
-      if (ctx.status) atomicCAS(ctx.status, 0, 0x100 + ctx.site);
-      return false;
-    }
+    if (globaltimer_ns() - t0 > ctx.limit_ns) return wait_gave_up(ctx);
   }
 }
 
@@ -216,11 +214,7 @@ __device__ bool grid_barrier(const SmallMArgs& a, const WaitCtx& ctx) {
   const uint64_t t0 = globaltimer_ns();
   while (ld_acquire(a.bar_gen) == g0) {
     __nanosleep(100);
-    if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
-      *ctx.abort_flag = 1;
-      if (ctx.status) atomicCAS(ctx.status, 0, 0x100 + ctx.site);
-      return false;
-    }
+    if (globaltimer_ns() - t0 > ctx.limit_ns) return wait_gave_up(ctx);
   }
   return true;
 }
@@ -249,6 +243,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* afull = lempty + kLoraSlots;
   uint64_t* accfull = afull + L::kASlots;
   uint64_t* accempty = accfull + 2;
+  uint64_t* mma_drain = accempty + 2;  // an issuer's MMAs ended (abort)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::offSlot);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::offAbort);
 
@@ -278,6 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&accfull[b], I);
       mbar_init(&accempty[b], 4);
     }
+    for (int i = 0; i < 4; ++i) mbar_init(&mma_drain[i], 1);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -308,7 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // producer 0 also issues every T and LoRA unit.
     const int p = warp == 0 ? 0 : warp - kProducerWarp1 + 1;
     if (lane == 0) {
-      const WaitCtx ctx{abort_flag, args.status, 41};
+      const WaitCtx ctx{abort_flag, args.status, 41, args.wait_ns};
       int jm = 0, jl = 0;
       bool ok = true;
       auto lora_slot = [&](uint8_t*& dst) -> uint64_t* {
@@ -362,15 +358,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (*abort_flag) {
         // Let the copies this thread issued land before the CTA exits.
-        const uint64_t t0 = globaltimer_ns();
         for (int i = (jm > S ? jm - S : 0); i < jm; ++i)
-          if (i % kProducers == p)
-            while (!mbar_try_wait(&full[i % S], (i / S) & 1) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
-            }
+          if (i % kProducers == p) mbar_drain(&full[i % S], (i / S) & 1);
         for (int i = (jl > kLoraSlots ? jl - kLoraSlots : 0); i < jl; ++i)
-          while (!mbar_try_wait(&lfull[i % kLoraSlots], (i / kLoraSlots) & 1) &&
-                 globaltimer_ns() - t0 < kWaitTimeoutNs) {
-          }
+          mbar_drain(&lfull[i % kLoraSlots], (i / kLoraSlots) & 1);
       }
     }
   } else if (((warp >= 1 && warp <= 3) || warp == kIssuerWarp3) && (warp == kIssuerWarp3 ? 3 : warp - 1) < I) {
@@ -380,7 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // unit.  All issuers commit to accfull at each segment's end.
     const int iss = warp == kIssuerWarp3 ? 3 : warp - 1;
     if (lane == 0) {
-      const WaitCtx ctx{abort_flag, args.status, 42};
+      const WaitCtx ctx{abort_flag, args.status, 42, args.wait_ns};
       const uint32_t idesc_main = idesc_bf16_f32(kTileRows, MP, false, false);
       const uint32_t idesc_smem = idesc_bf16_f32(kTileRows, MP, true, false);  // A^T / B^T tile, MN-major
       int jm = 0, jl = 0, seg = 0;
@@ -460,10 +451,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int lk = 0; lk < args.L && ok; ++lk) smem_unit(d, lk == 0);
         end_seg();
       }
+      if (!ok) {
+        // Aborted: the MMAs this thread issued end before TMEM is freed.
+        umma_commit(&mma_drain[iss]);
+        mbar_drain(&mma_drain[iss], 0);
+      }
     }
   } else if (warp >= 4 && warp < 8) {
     // ------------------------------------------------------------ epilogue
-    const WaitCtx ctx{abort_flag, args.status, 43};
+    const WaitCtx ctx{abort_flag, args.status, 43, args.wait_ns};
     const int q = warp & 3;
     const int row = q * 32 + lane;  // accumulator lane: weight row of the tile, or rank index j
     const int G4 = args.G4;
@@ -589,7 +585,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // block constants of a unit are loaded kPrefetch own units ahead into a
     // register queue (the loop is unrolled so the queue stays in registers).
     // Unit positions advance by increments: no division in the loop.
-    const WaitCtx ctx{abort_flag, args.status, 44};
+    const WaitCtx ctx{abort_flag, args.status, 44, args.wait_ns};
     const int grp = (warp - kDecWarp0) >> 2;
     const int q = warp & 3;
     const int nl = q * 32 + lane;
@@ -724,7 +720,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // threads sums (tile, token group) items: the tile's weight ranges in CTA
   // order, then its LoRA part.
   if (threadIdx.x == 0) {
-    const WaitCtx ctx{abort_flag, args.status, 45};
+    const WaitCtx ctx{abort_flag, args.status, 45, args.wait_ns};
     const bool ok = !*abort_flag && grid_barrier(args, ctx);
     *abort_flag = ok ? 0 : 1;
   }
@@ -883,6 +879,7 @@ cudaError_t launch_small_m_fwd(const uint16_t* X, const uint8_t* codes, const ui
   a.t_l1 = reinterpret_cast<float*>(ws + wp.t_l1);
   a.partial = reinterpret_cast<float*>(ws + wp.partial);
   a.status = status;
+  a.wait_ns = wait_limit_ns();
   a.nf4 = P;
   switch (MP) {
     case 16: return launch_mp<16>(mC, mX, mA, mB, mT, a, stream);

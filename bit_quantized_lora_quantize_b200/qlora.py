@@ -35,6 +35,8 @@ _SIGS = {
                                                 ctypes.c_float, _P, _P, _P]),
     "qlora_workspace_bytes": (ctypes.c_size_t, [_I64, _I64, _I64, ctypes.c_int32]),
     "qlora_check_status": (ctypes.c_int, [_P, _P]),
+    "qlora_set_wait_timeout": (ctypes.c_int, [ctypes.c_uint64]),
+    "qlora_get_wait_timeout": (ctypes.c_uint64, []),
     "qlora_nf4_codebook": (None, [ctypes.POINTER(ctypes.c_float)]),
     "qlora_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "qlora_last_cuda_error": (ctypes.c_char_p, []),
@@ -226,9 +228,20 @@ def qlora_linear_bwd(dY: torch.Tensor, X: torch.Tensor, T_save: torch.Tensor, W:
     return dX, dA, dB
 
 
-def qlora_check_status(workspace: torch.Tensor) -> int:
-    """Synchronise and return the device status code (0 = OK, 6 = a pipeline wait timed out)."""
-    return int(lib().qlora_check_status(_ptr(workspace), _stream()))
+def qlora_check_status(workspace: torch.Tensor | None = None) -> int:
+    """Synchronise and return the device status code (0 = OK, 6 = a pipeline
+    wait timed out): the workspace's word (if given) and the library's own
+    words for the calls without a workspace."""
+    return int(lib().qlora_check_status(_ptr(workspace) if workspace is not None else None, _stream()))
+
+
+def qlora_set_wait_timeout(timeout_ns: int) -> None:
+    """Limit of every bounded wait in the kernels (0 = the default, 2 s)."""
+    _check("qlora_set_wait_timeout", lib().qlora_set_wait_timeout(int(timeout_ns)))
+
+
+def qlora_get_wait_timeout() -> int:
+    return int(lib().qlora_get_wait_timeout())
 
 
 def qlora_profile_start() -> None:
@@ -252,4 +265,4 @@ def qlora_profile_stop(max_entries: int = 32) -> dict:
 __all__ = ["qlora_profile_start", "qlora_profile_stop", "LIB_PATH", "lib", "QloraError", "PackedNF4", "packed_sizes", "qlora_nf4_codebook", "qlora_quantize_nf4",
            "qlora_dequantize_nf4", "qlora_workspace_bytes", "new_workspace", "qlora_linear_fwd", "qlora_linear_bwd",
            "qlora_linear_fwd_noalloc",
-           "qlora_check_status"]
+           "qlora_check_status", "qlora_set_wait_timeout", "qlora_get_wait_timeout"]

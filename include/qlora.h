@@ -167,7 +167,9 @@ QLORA_API qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, c
  * counterpart to this call; it exists for those callers only.
  *   Same arguments, outputs and supported shapes as qlora_linear_fwd, minus
  *   workspace/ws_bytes; the results agree with qlora_linear_fwd to within
- *   float32 summation order (for M <= 128 the two use different kernels).
+ *   float32 summation order: for every M this call runs the pair GEMM of the
+ *   large-M forward, while qlora_linear_fwd takes the weight-streaming kernel
+ *   for M <= 128.
  *   The call allocates nothing:
  *   its scratch is one fixed 16 MiB device array inside this library, which
  *   every GPU that loads the library keeps until the process exits.
@@ -182,9 +184,10 @@ QLORA_API qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, c
  *   - All calls on a device share the array.  Calls that may overlap on the
  *     GPU (other streams, or host threads without ordering) race and must be
  *     serialised by the caller.
- *   - Each call clears the status word and counters it uses; a pipeline
- *     timeout inside this call is not reported (qlora_check_status needs a
- *     workspace).
+ *   - Each call clears the counters it uses.  A pipeline wait that gives up
+ *     sets the array's status word, which stays set until
+ *     qlora_check_status(NULL, stream) (or with any workspace) on that device
+ *     reports QLORA_ERR_TIMEOUT and clears it.
  *   - For M > 128 it runs the same GEMM launch as qlora_linear_fwd and gives
  *     the same bits.
  */
@@ -197,11 +200,24 @@ QLORA_API qlora_status qlora_linear_fwd_noalloc(const uint16_t* X, int64_t M, in
  * (0 for an unsupported shape). */
 QLORA_API size_t qlora_workspace_bytes(int64_t M, int64_t K, int64_t N, int32_t r);
 
-/* Synchronises `stream`, then reads the status word at the start of
- * `workspace`: QLORA_OK, or QLORA_ERR_TIMEOUT if a kernel of an earlier call
- * gave up on a pipeline wait (its outputs are then undefined).  The word is
- * reset to zero. */
+/* Synchronises `stream`, then reads the status words: the one at the start
+ * of `workspace` (skipped when workspace is NULL) and the two the library
+ * keeps on the current device for calls that take no workspace
+ * (qlora_quantize_nf4 and qlora_linear_fwd_noalloc).  Returns QLORA_OK, or
+ * QLORA_ERR_TIMEOUT if a kernel of an earlier call gave up on a pipeline wait
+ * (its outputs are then undefined).  Every word read is reset to zero. */
 QLORA_API qlora_status qlora_check_status(void* workspace, void* stream);
+
+/* Limit of every bounded wait inside the kernels (a pipeline barrier, a
+ * count another thread block raises, a grid barrier), in nanoseconds; 0
+ * restores the default of 2 s.  A wait that reaches the limit makes its
+ * kernel stop waiting, let its own copies and tensor-core work end, free its
+ * tensor memory and exit; qlora_check_status then reports QLORA_ERR_TIMEOUT.
+ * Applies to launches made after the call, from any host thread.  Limits
+ * above 60 s return QLORA_ERR_INVALID_ARG.  No counterpart on the pages:
+ * failure handling of this library. */
+QLORA_API qlora_status qlora_set_wait_timeout(uint64_t timeout_ns);
+QLORA_API uint64_t qlora_get_wait_timeout(void);
 
 /* The 16 NF4 levels (float32, ascending) this library encodes against. */
 QLORA_API void qlora_nf4_codebook(float out[16]);
