@@ -1,19 +1,33 @@
 """Benchmark of the frozen-NF4 LoRA linear layer on B200.
 
-One step = the whole hot path on one batch: NF4 quantization of the frozen
-weight (with double-quantized constants), the forward (T = s X A and the
-fused dequant-GEMM Y = X W'^T + T B) and the backward (U, dB, the fused
-dequant-GEMM dX = dY W' + U A^T, dA), through the C ABI of libqlora.so.
+One step = the whole hot path on one batch of a LLaMA-65B-shaped block:
+the one-shot NF4 quantization (with double-quantized constants) of the
+block's seven frozen weights (q, k, v, o 8192 x 8192; gate, up 22016 x 8192;
+down 8192 x 22016; 809.5 M parameters, 2.04 GB read and written), then the
+forward of the seven LoRA linears (T = s X A and the fused dequant-GEMM
+Y = X W'^T + T B) and their backward (U, dB, the fused dequant-GEMM
+dX = dY W' + U A^T, dA), 4096 tokens, r = 64, scale 0.25, seeded synthetic
+inputs, all through the C ABI of libqlora.so.  This is the headline `value`
+(TFLOP/s of the algorithmic fwd+bwd work over the whole step time,
+quantization included) with tokens/s beside it.
 
-Workload (N = 1): the LLaMA-7B attention projection, W 4096 x 4096 bf16
-~N(0, 0.02^2) with 0.1% of entries x10, 4096 tokens, r = 64, scale 0.25,
-seeded synthetic data.  With --gpus N (torchrun, one process per GPU) every
-rank runs its own batch of 4096 tokens (weak scaling) and the adapter
-gradients dA, dB are summed over ranks with one NCCL all-reduce per step
-(the data-parallel exchange).
+The same JSON line carries, as nested objects measured the same way:
+  mlp_trio   LLaMA-7B MLP (gate, up 11008 x 4096; down 4096 x 11008),
+             8192 tokens, SiLU-gated, fwd+bwd through the three linears
+             (weights quantized once, outside the step);
+  attn_proj  LLaMA-7B attention projection 4096^2 with 0.1 % outliers,
+             4096 tokens, quantize + fwd + bwd;
+  small_m    the small-M forward sweep (M in {1, 4, 16, 64}) as NF4 weight
+             GB/s against the HBM peak.
+
+With --gpus N every rank runs its own 4096 tokens through the block (weak
+scaling) and the adapter gradients of the seven linears, written by the
+backward into one flat bucket, are summed over ranks by one NCCL all-reduce
+per step (the data-parallel exchange).  Run without torchrun, --gpus N > 1
+re-launches itself under torch.distributed.run with N processes.
 
 Prints one JSON line (rank 0).  `--impl reference` times the CPU oracle (the
-float64 restatement in oracle/) on a bounded sample of the same workload.
+float64 restatement in oracle/) on a bounded sample of the block step.
 """
 
 from __future__ import annotations
@@ -21,6 +35,7 @@ from __future__ import annotations
 import argparse
 import json
 import os
+import socket
 import subprocess
 import sys
 import tempfile
@@ -31,8 +46,12 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "QLoRA linear fwd+bwd TFLOP/s & tokens/s; small-M NF4 weight GB/s vs HBM peak"
-WORKLOAD = dict(workload="llama7b_attn_proj_qlora_linear", M=4096, K=4096, N=4096, r=64, scale=0.25,
-                outliers="0.1% x10", step="quantize_nf4 + linear_fwd + linear_bwd")
+M_BLOCK, R, SCALE = 4096, 64, 0.25
+BLOCK_WORKLOAD = dict(
+    workload="llama65b_block_linears", M=M_BLOCK, r=R, scale=SCALE,
+    linears="q,k,v,o 8192x8192; gate,up 22016x8192; down 8192x22016 (out x in)",
+    step="quantize_nf4 x7 (one-shot, 809.5M params) + linear_fwd x7 + linear_bwd x7")
+L2_NOTE = "flushed between timed steps (256 MB write)"
 
 
 def flops_fwd(M, K, N, r):
@@ -43,6 +62,17 @@ def flops_bwd(M, K, N, r):
     return 2 * M * N * K + 4 * M * r * (K + N)
 
 
+def nf4_bytes(numel):
+    """Packed bytes of a weight: codes, 8-bit constants, float group maxima."""
+    nb = -(-numel // 64)
+    return (numel + 1) // 2 + nb + 4 * (-(-nb // 256))
+
+
+def quantize_bytes(numel):
+    """Algorithmic HBM bytes of one quantization: bf16 in, packed out."""
+    return 2 * numel + nf4_bytes(numel)
+
+
 def load_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -51,6 +81,13 @@ def load_peaks():
                     bf16_tflops_sustained=float(p["bf16_tflops_sustained"]), source="measured")
     except Exception:
         return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
 
 
 class ClockSampler:
@@ -157,71 +194,93 @@ class ClockSampler:
                 "samples": len(rows), "source": "nvidia-smi"}
 
 
-def cpu_oracle_sample(budget_rows: int = 1024):
-    """Time the oracle on a bounded sample of the workload: quantize the whole
-    4096 x 4096 weight, then forward + backward on `budget_rows` token rows."""
+# ---------------------------------------------------------------- CPU oracle
+def cpu_oracle_block_sample(rows: int = 128, slab: int = 128):
+    """Time the float64 oracle on a bounded sample of the block step and
+    scale it to the whole step.
+
+    Sample: for each of the seven linears, the quantization of a `slab`-row
+    slab of its weight (slab x K of the N x K weight) and the forward +
+    backward of `rows` tokens against that slab.  The whole step's time is
+    estimated as (sampled quantize time) x (809.5 M / sampled parameters) +
+    (sampled fwd+bwd time) x (step flops / sampled flops)."""
     import numpy as np
     from bit_quantized_lora_quantize_b200 import synthetic
     from oracle import dequantize_nf4, lora_linear_backward, lora_linear_forward, quantize_nf4
 
-    case = synthetic.attn_proj_case()
-    M, K, N, r = budget_rows, case.K, case.N, case.r
-    W = case.W.float().numpy()
-    X = case.X[:M].double().numpy()
-    dY = case.dY[:M].double().numpy()
-    A = case.A.double().numpy()
-    B = case.B.double().numpy()
-    t0 = time.perf_counter()
-    codes, aq, sc = quantize_nf4(W)
-    Wdq = dequantize_nf4(codes, aq, sc, W.size).reshape(N, K)
-    lora_linear_forward(X, Wdq, A, B, case.scale)
-    lora_linear_backward(dY, X, Wdq, A, B, case.scale)
-    dt = time.perf_counter() - t0
-    fl = flops_fwd(M, K, N, r) + flops_bwd(M, K, N, r)
+    rng = np.random.default_rng(5)
+    t_q = t_g = 0.0
+    p_s = fl_s = 0
+    p_full = fl_full = 0
+    for i, (name, N, K) in enumerate(synthetic.LLAMA65B_LINEARS):
+        W = synthetic.weight_only(slab, K, seed=300 + i).float().numpy()
+        X = rng.standard_normal((rows, K))
+        dY = rng.standard_normal((rows, slab))
+        A = rng.standard_normal((K, R)) * 0.01
+        B = rng.standard_normal((R, slab)) * 0.01
+        t0 = time.perf_counter()
+        codes, aq, sc = quantize_nf4(W)
+        t1 = time.perf_counter()
+        Wdq = dequantize_nf4(codes, aq, sc, W.size).reshape(slab, K)
+        lora_linear_forward(X, Wdq, A, B, SCALE)
+        lora_linear_backward(dY, X, Wdq, A, B, SCALE)
+        t2 = time.perf_counter()
+        t_q += t1 - t0
+        t_g += t2 - t1
+        p_s += W.size
+        fl_s += flops_fwd(rows, K, slab, R) + flops_bwd(rows, K, slab, R)
+        p_full += N * K
+        fl_full += flops_fwd(M_BLOCK, K, N, R) + flops_bwd(M_BLOCK, K, N, R)
+    step_s = t_q * p_full / p_s + t_g * fl_full / fl_s
     try:
         from threadpoolctl import threadpool_info
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+        blas = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
     except Exception:
-        cores = os.cpu_count() or 1
-    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": int(cores), "kind": "oracle",
-            "sample": f"quantize of the full 4096x4096 weight + fwd+bwd on {M} of 4096 token rows (float64 numpy)",
-            "seconds": dt, "tokens_per_s": M / dt}
+        blas = None
+    return {"value": fl_full / step_s / 1e12, "unit": "TFLOP/s", "cores": host_cores(), "blas_threads": blas,
+            "kind": "oracle",
+            "sample": (f"per linear: quantize of a {slab}-row slab of the weight + fwd+bwd of {rows} tokens "
+                       f"against it (float64 numpy); whole-step time scaled from the sample by parameter "
+                       f"count (quantize) and by flops (fwd+bwd)"),
+            "sample_seconds": t_q + t_g, "est_step_seconds": step_s, "tokens_per_s": M_BLOCK / step_s,
+            "quantize_mparams_per_s": p_s / t_q / 1e6, "fwd_bwd_gflops": fl_s / t_g / 1e9}
+
+
+def block_flops():
+    from bit_quantized_lora_quantize_b200 import synthetic
+    return sum(flops_fwd(M_BLOCK, K, N, R) + flops_bwd(M_BLOCK, K, N, R) for _, N, K in synthetic.LLAMA65B_LINEARS)
 
 
 def run_reference(args, rank, world):
     if rank != 0:
         return
-    vals = []
     for _ in range(args.warmup):
-        cpu_oracle_sample(256)
-    samples = []
-    for _ in range(args.steps):
-        s = cpu_oracle_sample(512)
-        samples.append(s)
-        vals.append(s["value"])
-    v = sorted(vals)[len(vals) // 2]
+        cpu_oracle_block_sample(rows=16, slab=64)
+    samples = [cpu_oracle_block_sample(rows=128, slab=128) for _ in range(args.steps)]
+    vals = sorted(s["value"] for s in samples)
+    v = vals[len(vals) // 2]
     cb = dict(samples[-1])
     cb["value"] = v
-    # The whole step's flops at the sample's rate: the time one full step would take.
-    M, K, N, r = WORKLOAD["M"], WORKLOAD["K"], WORKLOAD["N"], WORKLOAD["r"]
-    ms_full = (flops_fwd(M, K, N, r) + flops_bwd(M, K, N, r)) / (v * 1e12) * 1e3
+    ms_full = block_flops() / (v * 1e12) * 1e3
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_full, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": dict(WORKLOAD), "cpu_baseline": cb, "tokens_per_s": M / (ms_full * 1e-3),
+            "config": dict(BLOCK_WORKLOAD, l2="n/a (host)"), "cpu_baseline": cb,
+            "tokens_per_s": M_BLOCK / (ms_full * 1e-3),
             "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
-def traffic_for(kernel: str):
+# ---------------------------------------------------------------- timing helpers
+def traffic_for(key: str):
     """DRAM bytes per launch from the committed ncu summary, if it still
-    describes the current kernel source."""
+    describes the current kernel source (else None)."""
     import hashlib
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             t = json.load(f)
-        ent = t[kernel]
+        ent = t[key]
         hsh = hashlib.sha256()
         for name in ent["sources"]:  # the kernel's .cu file and the headers it includes
             with open(os.path.join(ROOT, "bit_quantized_lora_quantize_b200", "csrc", name), "rb") as f:
@@ -233,6 +292,382 @@ def traffic_for(kernel: str):
         return None
 
 
+class Calls:
+    """Runs the library calls of a step.  Each call is exactly one kernel
+    launch; in profiling mode a pair of CUDA events on the launching stream
+    brackets every call, keyed by (kernel, linear)."""
+
+    def __init__(self):
+        self.recs = None
+
+    def __call__(self, kernel, tag, work, fn):
+        if self.recs is None:
+            return fn()
+        import torch
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        out = fn()
+        b.record()
+        self.recs.append((kernel, tag, work, a, b))
+        return out
+
+    def profile(self, step, n, flush):
+        """Run `n` more steps with per-call events; return
+        {(kernel, tag): dict(ms_total, launches, work)} and the launch count."""
+        import torch
+        self.recs = []
+        for _ in range(n):
+            flush.zero_()
+            step()
+        torch.cuda.synchronize()
+        agg = {}
+        for kernel, tag, work, a, b in self.recs:
+            e = agg.setdefault((kernel, tag), {"ms_total": 0.0, "launches": 0, "work": work})
+            e["ms_total"] += a.elapsed_time(b)
+            e["launches"] += 1
+        self.recs = None
+        return agg
+
+
+def time_steps(step, steps, flush, world, local_rank, sample_clocks=True):
+    """Device time of exactly `steps` steps (CUDA events around each step on
+    the launching stream, L2 flushed before each), max over ranks."""
+    import torch
+    import torch.distributed as dist
+    stream = torch.cuda.current_stream()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    sampler = ClockSampler(local_rank) if sample_clocks else None
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+    for i in range(steps):
+        flush.zero_()
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if sampler else None
+    total = sum(a.elapsed_time(b) for a, b in evs)
+    t = torch.tensor([total], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item()) / steps, clocks
+
+
+def time_e2e(e2e_step, steps, world):
+    """Device time per step of the end-to-end step (host copies included)."""
+    import torch
+    import torch.distributed as dist
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item()) / steps
+
+
+def kernel_table(agg):
+    tot = sum(v["ms_total"] for v in agg.values()) or 1.0
+    out = {}
+    for (kernel, tag), v in sorted(agg.items()):
+        out[f"{kernel}/{tag}"] = {"us_per_launch": v["ms_total"] * 1e3 / v["launches"], "launches": v["launches"],
+                                  "share": v["ms_total"] / tot}
+    return out
+
+
+def gemm_roofline(agg, peaks, sustained=False):
+    """Roofline of the dominant fused GEMM (largest total time over the
+    profiled steps): algorithmic flops per launch / mean launch time, against
+    the measured bf16 peak: the sustained figure for kernels timed inside a
+    long step (power-capped clocks), the burst figure otherwise."""
+    gem = {k: v for k, v in agg.items() if k[0].startswith("fused_nf4")}
+    if not gem:
+        return None
+    key = max(gem, key=lambda k: gem[k]["ms_total"])
+    v = gem[key]
+    ms = v["ms_total"] / v["launches"]
+    achieved = v["work"]["flops"] / (ms * 1e-3) / 1e12
+    tkey = f"{key[0]}/{key[1]}"
+    peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+    kind = "sustained" if sustained else "burst"
+    return {"bound": "tensor", "kernel": tkey, "achieved": achieved, "peak": peak,
+            "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic_for(tkey),
+            "peak_source": f"{peaks['source']} bf16 {kind} ({'of measured' if peaks['source'] == 'measured' else 'of fallback'})",
+            "frac_of_burst": achieved / peaks["bf16_tflops"],
+            "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"], "us_per_launch": ms * 1e3,
+            "flops_per_launch": v["work"]["flops"],
+            "flops_counted": "2MNK + 2Mr(N+K) (dense product, LoRA product and the rank-r intermediate)"}
+
+
+def quantize_roofline(agg, peaks):
+    qk = {k: v for k, v in agg.items() if k[0] == "quantize_nf4"}
+    if not qk:
+        return None
+    by = sum(v["work"]["bytes"] * v["launches"] for v in qk.values())
+    ms = sum(v["ms_total"] for v in qk.values())
+    steps = max(v["launches"] for v in qk.values())
+    achieved = by / (ms * 1e-3) / 1e9
+    return {"bound": "hbm", "kernel": "quantize_nf4", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / peaks["hbm_gbs"], "traffic": traffic_for("quantize_nf4/gate"),
+            "traffic_note": "per launch, for the 22016 x 8192 weight (one of the seven)",
+            "bytes_per_step": by / steps, "us_per_step": ms * 1e3 / steps,
+            "bytes_counted": "2 B read + 0.5159 B written per weight",
+            "peak_source": f"{peaks['source']} HBM copy bandwidth"}
+
+
+# ---------------------------------------------------------------- the block step
+class Linear:
+    """Device-resident tensors of one LoRA linear (inputs, outputs, workspace)."""
+
+    def __init__(self, q, case, tag, dev, grads=None):
+        import torch
+        self.tag = tag
+        self.case = case
+        self.M, self.K, self.N, self.r, self.s = case.M, case.K, case.N, case.r, case.scale
+        self.W = case.W.to(dev)
+        self.P = q.qlora_quantize_nf4(self.W)
+        self.A, self.B, self.dY = case.A.to(dev), case.B.to(dev), case.dY.to(dev)
+        self.ws = q.new_workspace(self.M, self.K, self.N, self.r, dev)
+        self.Y = torch.empty(self.M, self.N, dtype=torch.bfloat16, device=dev)
+        self.T = torch.empty(self.M, self.r, dtype=torch.float32, device=dev)
+        self.dX = torch.empty(self.M, self.K, dtype=torch.bfloat16, device=dev)
+        if grads is None:
+            self.dA = torch.empty(self.K, self.r, dtype=torch.float32, device=dev)
+            self.dB = torch.empty(self.r, self.N, dtype=torch.float32, device=dev)
+        else:
+            self.dA, self.dB = grads
+
+    @property
+    def numel(self):
+        return self.N * self.K
+
+
+def make_block(q, synthetic, dev, rank, grads_bucket_cls):
+    import torch
+    cases = synthetic.llama65b_block(M_BLOCK, R, SCALE)
+    if rank != 0:
+        # Other ranks take other tokens (and upstream gradients): weak scaling.
+        g = torch.Generator().manual_seed(1000 + rank)
+        X = (torch.randn(cases[0][1].X.shape, generator=g)).to(torch.bfloat16)
+        Xd = (torch.randn(cases[-1][1].X.shape, generator=g)).to(torch.bfloat16)
+        for _, c in cases:
+            c.X = X if c.K == 8192 else Xd
+            c.dY = torch.randn(c.dY.shape, generator=g).to(torch.bfloat16)
+    bucket = grads_bucket_cls([(c.K, c.N, c.r) for _, c in cases], dev)
+    X = cases[0][1].X.to(dev)
+    Xd = cases[-1][1].X.to(dev)
+    lins = []
+    for i, (name, c) in enumerate(cases):
+        lin = Linear(q, c, name, dev, grads=bucket[i])
+        lin.X = X if c.K == 8192 else Xd
+        lins.append(lin)
+    return lins, bucket, X, Xd
+
+
+def block_step_fn(q, lins, calls, bucket, world):
+    def step():
+        for l in lins:
+            calls("quantize_nf4", l.tag, {"bytes": quantize_bytes(l.numel)},
+                  lambda l=l: q.qlora_quantize_nf4(l.W, out=l.P))
+        for l in lins:
+            calls("fused_nf4_fwd", l.tag, {"flops": 2 * l.M * l.N * l.K + 2 * l.M * l.r * (l.N + l.K)},
+                  lambda l=l: q.qlora_linear_fwd(l.X, l.P, l.A, l.B, l.s, workspace=l.ws, Y=l.Y, T_save=l.T))
+        for l in reversed(lins):
+            calls("fused_nf4_dx", l.tag, {"flops": 2 * l.M * l.N * l.K + 2 * l.M * l.r * (l.N + l.K)},
+                  lambda l=l: q.qlora_linear_bwd(l.dY, l.X, l.T, l.P, l.A, l.B, l.s, workspace=l.ws, dX=l.dX,
+                                                 dA=l.dA, dB=l.dB))
+        if world > 1:
+            bucket.all_reduce()
+    return step
+
+
+def bench_block(args, q, synthetic, dp, dev, rank, world, local_rank, flush, peaks):
+    import torch
+    lins, bucket, X, Xd = make_block(q, synthetic, dev, rank, dp.GradBucket)
+    calls = Calls()
+    step = block_step_fn(q, lins, calls, bucket, world)
+    fl_step = sum(flops_fwd(l.M, l.K, l.N, l.r) + flops_bwd(l.M, l.K, l.N, l.r) for l in lins)
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    for l in lins:
+        if q.qlora_check_status(l.ws) != 0:
+            raise RuntimeError("device pipeline timeout during warm-up")
+    ms, clocks = time_steps(step, args.steps, flush, world, local_rank)
+    agg = calls.profile(step, args.steps, flush)
+
+    # End to end through the public API: every step copies the seven bf16
+    # weights, both inputs and the seven dY in from pinned host memory, and
+    # the seven Y and dX and the gradient bucket back.
+    pin = lambda t: t.cpu().pin_memory()  # noqa: E731
+    hW = [pin(l.case.W) for l in lins]
+    hdY = [pin(l.case.dY) for l in lins]
+    hX, hXd = pin(lins[0].case.X), pin(lins[-1].case.X)
+    hY = [torch.empty(l.Y.shape, dtype=l.Y.dtype).pin_memory() for l in lins]
+    hdX = [torch.empty(l.dX.shape, dtype=l.dX.dtype).pin_memory() for l in lins]
+    hG = torch.empty(bucket.flat.shape, dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * 2 for t in hW + hdY) + hX.numel() * 2 + hXd.numel() * 2
+    d2h = sum(t.numel() * 2 for t in hY + hdX) + hG.numel() * 4
+
+    def e2e_step():
+        for l, w, dy in zip(lins, hW, hdY):
+            l.W.copy_(w, non_blocking=True)
+            l.dY.copy_(dy, non_blocking=True)
+        X.copy_(hX, non_blocking=True)
+        Xd.copy_(hXd, non_blocking=True)
+        step()
+        for l, y, dx in zip(lins, hY, hdX):
+            y.copy_(l.Y, non_blocking=True)
+            dx.copy_(l.dX, non_blocking=True)
+        hG.copy_(bucket.flat, non_blocking=True)
+
+    e2e_ms = time_e2e(e2e_step, args.steps, world)
+    for l in lins:
+        if q.qlora_check_status(l.ws) != 0:
+            raise RuntimeError("device pipeline timeout during timing")
+    launches_per_step = 3 * len(lins)
+    res = {
+        "ms_per_step": ms, "value": fl_step * world / (ms * 1e-3) / 1e12,
+        "tokens_per_s": M_BLOCK * world / (ms * 1e-3),
+        "tflops_dense_only": sum(4 * l.M * l.N * l.K for l in lins) * world / (ms * 1e-3) / 1e12,
+        "flops_per_step": fl_step, "clocks": clocks, "kernels": kernel_table(agg),
+        "roofline": gemm_roofline(agg, peaks, sustained=True), "roofline_quantize": quantize_roofline(agg, peaks),
+        "gpu_launches": launches_per_step * args.steps,
+        "e2e": {"value": fl_step * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                "copies": "in: 7 bf16 weights, X, X_down, 7 dY; out: 7 Y, 7 dX, dA|dB bucket"},
+        "grad_bucket_bytes": bucket.nbytes,
+    }
+    del lins, bucket, hW, hdY, hY, hdX
+    torch.cuda.empty_cache()
+    return res
+
+
+# ---------------------------------------------------------------- MLP trio
+def bench_trio(args, q, synthetic, dev, flush, peaks, local_rank):
+    import torch
+    t = synthetic.mlp_trio()
+    M, D, Fd, r, s = t.X.shape[0], t.X.shape[1], t.Wg.shape[0], t.Ag.shape[1], t.scale
+    d = lambda x: x.to(dev)  # noqa: E731
+    Pg, Pu, Pd = (q.qlora_quantize_nf4(d(w)) for w in (t.Wg, t.Wu, t.Wd))
+    X, dY = d(t.X), d(t.dY)
+    Ag, Au, Ad, Bg, Bu, Bd = (d(x) for x in (t.Ag, t.Au, t.Ad, t.Bg, t.Bu, t.Bd))
+    wsg, wsu = q.new_workspace(M, D, Fd, r, dev), q.new_workspace(M, D, Fd, r, dev)
+    wsd = q.new_workspace(M, Fd, D, r, dev)
+    bf = torch.bfloat16
+    G, Up = torch.empty(M, Fd, dtype=bf, device=dev), torch.empty(M, Fd, dtype=bf, device=dev)
+    Tg, Tu, Td = (torch.empty(M, r, dtype=torch.float32, device=dev) for _ in range(3))
+    Y = torch.empty(M, D, dtype=bf, device=dev)
+    dH = torch.empty(M, Fd, dtype=bf, device=dev)
+    H, dG, dU = (torch.empty(M, Fd, dtype=bf, device=dev) for _ in range(3))
+    dXg, dXu = torch.empty(M, D, dtype=bf, device=dev), torch.empty(M, D, dtype=bf, device=dev)
+    dX = torch.empty(M, D, dtype=bf, device=dev)
+    gA = [torch.empty(k, r, dtype=torch.float32, device=dev) for k in (D, D, Fd)]
+    gB = [torch.empty(r, n, dtype=torch.float32, device=dev) for n in (Fd, Fd, D)]
+    calls = Calls()
+    fl = lambda K, N: 2 * M * N * K + 2 * M * r * (N + K)  # noqa: E731
+
+    def step():
+        calls("fused_nf4_fwd", "gate", {"flops": fl(D, Fd)},
+              lambda: q.qlora_linear_fwd(X, Pg, Ag, Bg, s, workspace=wsg, Y=G, T_save=Tg))
+        calls("fused_nf4_fwd", "up", {"flops": fl(D, Fd)},
+              lambda: q.qlora_linear_fwd(X, Pu, Au, Bu, s, workspace=wsu, Y=Up, T_save=Tu))
+        calls("silu_gate_fwd", "trio", {"bytes": 3 * 2 * M * Fd}, lambda: q.qlora_silu_gate_fwd(G, Up, H))
+        calls("fused_nf4_fwd", "down", {"flops": fl(Fd, D)},
+              lambda: q.qlora_linear_fwd(H, Pd, Ad, Bd, s, workspace=wsd, Y=Y, T_save=Td))
+        calls("fused_nf4_dx", "down", {"flops": fl(Fd, D)},
+              lambda: q.qlora_linear_bwd(dY, H, Td, Pd, Ad, Bd, s, workspace=wsd, dX=dH, dA=gA[2], dB=gB[2]))
+        calls("silu_gate_bwd", "trio", {"bytes": 5 * 2 * M * Fd}, lambda: q.qlora_silu_gate_bwd(G, Up, dH, dG, dU))
+        calls("fused_nf4_dx", "gate", {"flops": fl(D, Fd)},
+              lambda: q.qlora_linear_bwd(dG, X, Tg, Pg, Ag, Bg, s, workspace=wsg, dX=dXg, dA=gA[0], dB=gB[0]))
+        calls("fused_nf4_dx", "up", {"flops": fl(D, Fd)},
+              lambda: q.qlora_linear_bwd(dU, X, Tu, Pu, Au, Bu, s, workspace=wsu, dX=dXu, dA=gA[1], dB=gB[1]))
+        torch.add(dXg, dXu, out=dX)  # the input's two gradient paths (torch add, bf16)
+
+    fl_step = 2 * (flops_fwd(M, D, Fd, r) + flops_bwd(M, D, Fd, r)) + flops_fwd(M, Fd, D, r) + flops_bwd(M, Fd, D, r)
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    ms, clocks = time_steps(step, args.steps, flush, 1, local_rank)
+    agg = calls.profile(step, args.steps, flush)
+    hX, hdY = t.X.pin_memory(), t.dY.pin_memory()
+    hY = torch.empty(Y.shape, dtype=bf).pin_memory()
+    hdX = torch.empty(M, D, dtype=bf).pin_memory()
+
+    def e2e_step():
+        X.copy_(hX, non_blocking=True)
+        dY.copy_(hdY, non_blocking=True)
+        step()
+        hY.copy_(Y, non_blocking=True)
+        hdX.copy_(dX, non_blocking=True)
+
+    e2e_ms = time_e2e(e2e_step, args.steps, 1)
+    for w in (wsg, wsu, wsd):
+        if q.qlora_check_status(w) != 0:
+            raise RuntimeError("device pipeline timeout (trio)")
+    res = {"workload": "llama7b_mlp_trio", "M": M, "D": D, "F": Fd, "r": r, "scale": s,
+           "step": "linear_fwd gate, up; silu_gate_fwd; linear_fwd down; linear_bwd down; silu_gate_bwd; "
+                   "linear_bwd gate, up; dX = dX_gate + dX_up (torch add) (weights quantized once, outside the step)",
+           "value": fl_step / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms,
+           "tokens_per_s": M / (ms * 1e-3), "clocks": clocks, "kernels": kernel_table(agg),
+           "roofline": gemm_roofline(agg, peaks, sustained=True), "gpu_launches": 8 * args.steps,
+           "e2e": {"value": fl_step / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                   "h2d_bytes_per_step": (hX.numel() + hdY.numel()) * 2,
+                   "d2h_bytes_per_step": (hY.numel() + hdX.numel()) * 2, "ms_per_step": e2e_ms},
+           "l2": L2_NOTE}
+    torch.cuda.empty_cache()
+    return res
+
+
+# ---------------------------------------------------------------- attention projection
+def bench_attn(args, q, synthetic, dev, flush, peaks, local_rank):
+    import torch
+    case = synthetic.attn_proj_case()
+    lin = Linear(q, case, "attn_proj", dev)
+    lin.X = case.X.to(dev)
+    calls = Calls()
+    fl = 2 * lin.M * lin.N * lin.K + 2 * lin.M * lin.r * (lin.N + lin.K)
+
+    def step():
+        calls("quantize_nf4", "attn_proj", {"bytes": quantize_bytes(lin.numel)},
+              lambda: q.qlora_quantize_nf4(lin.W, out=lin.P))
+        calls("fused_nf4_fwd", "attn_proj", {"flops": fl},
+              lambda: q.qlora_linear_fwd(lin.X, lin.P, lin.A, lin.B, lin.s, workspace=lin.ws, Y=lin.Y, T_save=lin.T))
+        calls("fused_nf4_dx", "attn_proj", {"flops": fl},
+              lambda: q.qlora_linear_bwd(lin.dY, lin.X, lin.T, lin.P, lin.A, lin.B, lin.s, workspace=lin.ws,
+                                         dX=lin.dX, dA=lin.dA, dB=lin.dB))
+
+    fl_step = flops_fwd(lin.M, lin.K, lin.N, lin.r) + flops_bwd(lin.M, lin.K, lin.N, lin.r)
+    for _ in range(max(3, args.warmup)):
+        step()
+    ms, _ = time_steps(step, args.steps, flush, 1, local_rank, sample_clocks=False)
+    agg = calls.profile(step, args.steps, flush)
+    if q.qlora_check_status(lin.ws) != 0:
+        raise RuntimeError("device pipeline timeout (attn_proj)")
+    res = {"workload": "llama7b_attn_proj_qlora_linear", "M": lin.M, "K": lin.K, "N": lin.N, "r": lin.r,
+           "outliers": "0.1% x10", "step": "quantize_nf4 + linear_fwd + linear_bwd",
+           "value": fl_step / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms,
+           "tokens_per_s": lin.M / (ms * 1e-3), "kernels": kernel_table(agg), "roofline": gemm_roofline(agg, peaks)}
+    del lin
+    torch.cuda.empty_cache()
+    return res
+
+
+# ---------------------------------------------------------------- small-M sweep
 def small_m_sweep(q, synthetic, dev, flush, iters=10):
     """Small-M forward (W [N x 8192] NF4, M tokens, r = 64): NF4 weight bytes
     streamed per second, L2 flushed before every timed call."""
@@ -244,7 +679,7 @@ def small_m_sweep(q, synthetic, dev, flush, iters=10):
         W = synthetic.weight_only(N, 8192, seed=4).to(dev)
         Wp = q.qlora_quantize_nf4(W)
         del W
-        nf4_bytes = Wp.codes.numel() + Wp.absmax_q.numel() + 4 * Wp.absmax_scale.numel()
+        nb = nf4_bytes(N * 8192)
         for M in (1, 4, 16, 64):
             case = synthetic.small_m_case(M, N)
             X, A, B = (t.to(dev) for t in (case.X, case.A, case.B))
@@ -255,31 +690,25 @@ def small_m_sweep(q, synthetic, dev, flush, iters=10):
                 q.qlora_linear_fwd(X, Wp, A, B, 0.25, workspace=ws, Y=Y, T_save=T)
             stream = torch.cuda.current_stream()
             evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(iters)]
-            q.qlora_profile_start()
             for i in range(iters):
                 flush.zero_()
                 evs[i][0].record(stream)
                 q.qlora_linear_fwd(X, Wp, A, B, 0.25, workspace=ws, Y=Y, T_save=T)
                 evs[i][1].record(stream)
             torch.cuda.synchronize()
-            prof = q.qlora_profile_stop()
             us = sorted(a.elapsed_time(b) * 1e3 for a, b in evs)[iters // 2]
-            gbs = nf4_bytes / (us * 1e-6) / 1e9
-            ent = {"N": N, "K": 8192, "M": M, "us": us, "nf4_weight_gbs": gbs,
-                   "frac_hbm": gbs / peaks["hbm_gbs"], "nf4_bytes": nf4_bytes}
-            # The weight-streaming kernel alone (mean over the timed calls).
-            for name, (ms, calls, _) in prof.items():
-                if name in ("small_m_nf4_fwd", "fused_nf4_fwd"):
-                    k_us = ms * 1e3 / max(calls, 1)
-                    ent.update({"kernel": name, "kernel_us": k_us,
-                                "kernel_frac_hbm": nf4_bytes / (k_us * 1e-6) / 1e9 / peaks["hbm_gbs"]})
-            out.append(ent)
+            gbs = nb / (us * 1e-6) / 1e9
+            out.append({"N": N, "K": 8192, "M": M, "us": us, "nf4_weight_gbs": gbs,
+                        "frac_hbm": gbs / peaks["hbm_gbs"], "nf4_bytes": nb,
+                        "kernel": "small_m_nf4_fwd" if M <= 128 else "fused_nf4_fwd"})
+            if q.qlora_check_status(ws) != 0:
+                raise RuntimeError("device pipeline timeout (small M)")
     return out
 
 
+# ---------------------------------------------------------------- driver
 def run_ours(args, rank, world, local_rank):
     import torch
-    import torch.distributed as dist
 
     import bit_quantized_lora_quantize_b200 as q
     from bit_quantized_lora_quantize_b200 import build as qbuild, dp, synthetic
@@ -287,150 +716,49 @@ def run_ours(args, rank, world, local_rank):
     qbuild.build()
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    case = synthetic.attn_proj_case() if rank == 0 else synthetic.linear_case(
-        4096, 4096, 4096, 64, 0.25, 1 + 1000 * rank, outlier_frac=0.001)
-    M, K, N, r, s = case.M, case.K, case.N, case.r, case.scale
-    W = case.W.to(dev)
-    X, A, B, dY = (t.to(dev) for t in (case.X, case.A, case.B, case.dY))
-    ws = q.new_workspace(M, K, N, r, dev)
-    Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
-    T = torch.empty(M, r, dtype=torch.float32, device=dev)
-    dX = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
-    dA = torch.empty(K, r, dtype=torch.float32, device=dev)
-    dB = torch.empty(r, N, dtype=torch.float32, device=dev)
+    peaks = load_peaks()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # > L2 (126 MB)
-    reducer = dp.AdapterGradReducer(K, N, r, dev) if world > 1 else None
 
-    def step():
-        Wp = q.qlora_quantize_nf4(W)
-        q.qlora_linear_fwd(X, Wp, A, B, s, workspace=ws, Y=Y, T_save=T)
-        q.qlora_linear_bwd(dY, X, T, Wp, A, B, s, workspace=ws, dX=dX, dA=dA, dB=dB)
-        if reducer is not None:
-            reducer(dA, dB)
-        return Wp
-
-    for _ in range(max(3, args.warmup)):
-        step()
-    torch.cuda.synchronize()
-    if q.qlora_check_status(ws) != 0:
-        raise RuntimeError("device pipeline timeout during warm-up")
-
-    # ---------------- device-resident timing (kernels only), L2 flushed between steps
-    stream = torch.cuda.current_stream()
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    sampler = ClockSampler(local_rank)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    sampler.start()
-    for i in range(args.steps):
-        flush.zero_()
-        evs[i][0].record(stream)
-        step()
-        evs[i][1].record(stream)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    clocks = sampler.stop()
-    # Per-kernel durations (roofline, kernel table): the same K steps again
-    # with CUDA events recorded around every launch on the launching stream.
-    # Kept out of the timed steps above, because an event between two kernels
-    # stops the next one from starting before the previous one ends.
-    q.qlora_profile_start()
-    for i in range(args.steps):
-        flush.zero_()
-        step()
-    torch.cuda.synchronize()
-    prof = q.qlora_profile_stop()
-    step_ms = [a.elapsed_time(b) for a, b in evs]
-    total_ms = sum(step_ms)
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
-    ms_per_step = total_ms / args.steps
-    fl_step = flops_fwd(M, K, N, r) + flops_bwd(M, K, N, r)
-    value = fl_step * world / (ms_per_step * 1e-3) / 1e12
-    tokens_per_s = M * world / (ms_per_step * 1e-3)
-    # The same step time with only the dense products counted (4MNK: the
-    # frozen-weight GEMMs of forward and input gradient).
-    value_dense = 4 * M * N * K * world / (ms_per_step * 1e-3) / 1e12
-
-    # ---------------- end to end through the public API with host buffers
-    pin = lambda t: t.cpu().pin_memory()  # noqa: E731
-    hW, hX, hdY = pin(case.W), pin(case.X), pin(case.dY)
-    hdA = torch.empty(K, r, dtype=torch.float32).pin_memory()
-    hdB = torch.empty(r, N, dtype=torch.float32).pin_memory()
-    h2d = hW.numel() * 2 + hX.numel() * 2 + hdY.numel() * 2
-    d2h = hdA.numel() * 4 + hdB.numel() * 4
-
-    def e2e_step():
-        W.copy_(hW, non_blocking=True)
-        X.copy_(hX, non_blocking=True)
-        dY.copy_(hdY, non_blocking=True)
-        step()
-        hdA.copy_(dA, non_blocking=True)
-        hdB.copy_(dB, non_blocking=True)
-
-    for _ in range(2):
-        e2e_step()
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    t = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    e2e_ms = float(t.item()) / args.steps
-    e2e_value = fl_step * world / (e2e_ms * 1e-3) / 1e12
-    if q.qlora_check_status(ws) != 0:
-        raise RuntimeError("device pipeline timeout during timing")
-
-    small_m = small_m_sweep(q, synthetic, dev, flush) if (rank == 0 and not args.no_small_m) else None
-
+    blk = bench_block(args, q, synthetic, dp, dev, rank, world, local_rank, flush, peaks)
+    extra = rank == 0 and world == 1
+    trio = bench_trio(args, q, synthetic, dev, flush, peaks, local_rank) if extra and not args.block_only else None
+    attn = bench_attn(args, q, synthetic, dev, flush, peaks, local_rank) if extra and not args.block_only else None
+    small_m = small_m_sweep(q, synthetic, dev, flush) if (extra and not args.no_small_m) else None
     if rank != 0:
         return
-    peaks = load_peaks()
-    # Dominant kernel: the fused dequant-GEMM with the larger total time.
-    fused = {k: v for k, v in prof.items() if k.startswith("fused_nf4")}
-    dom = max(fused, key=lambda k: fused[k][0])
-    dom_ms = fused[dom][0] / fused[dom][1]
-    # Each fused launch also computes its rank-r intermediate (T = s X A in the
-    # forward, U = s dY B^T in the input gradient) besides the LoRA product.
-    dom_flops = 2 * M * N * K + 2 * M * r * (N + K)
-    achieved = dom_flops / (dom_ms * 1e-3) / 1e12
-    launches = sum(v[2] for v in prof.values())
-    kernels = {k: {"ms_per_call": v[0] / v[1], "calls": v[1], "share": v[0] / sum(x[0] for x in prof.values())}
-               for k, v in prof.items()}
-    cpu = cpu_oracle_sample(512) if (world == 1 and not args.no_cpu_baseline) else None
+    cpu = cpu_oracle_block_sample(rows=256, slab=256) if (world == 1 and not args.no_cpu_baseline) else None
     line = {
-        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-        "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": dict(WORKLOAD, parallelism=f"dp{world}", global_batch_tokens=M * world,
-                       l2="flushed between timed steps (256 MB write)"),
-        "tokens_per_s": tokens_per_s,
-        "tflops_dense_only": value_dense,
-        "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peaks["bf16_tflops"],
-                     "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": traffic_for(dom),
-                     "peak_source": f"{peaks['source']} bf16 burst", "ms_per_launch": dom_ms},
-        "kernels": kernels,
-        "gpu_launches": launches,
-        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": e2e_ms},
-        "clocks": clocks,
-        "cpu_baseline": cpu,
-        "small_m": small_m,
+        "metric": METRIC, "value": blk["value"], "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": blk["ms_per_step"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(BLOCK_WORKLOAD, parallelism=f"dp{world}", global_batch_tokens=M_BLOCK * world, l2=L2_NOTE),
+        "tokens_per_s": blk["tokens_per_s"], "tflops_dense_only": blk["tflops_dense_only"],
+        "flops_per_step": blk["flops_per_step"],
+        "roofline": blk["roofline"], "roofline_quantize": blk["roofline_quantize"],
+        "kernels": blk["kernels"], "gpu_launches": blk["gpu_launches"], "e2e": blk["e2e"],
+        "clocks": blk["clocks"], "cpu_baseline": cpu,
+        "grad_allreduce_bytes_per_step": blk["grad_bucket_bytes"] if world > 1 else 0,
+        "mlp_trio": trio, "attn_proj": attn, "small_m": small_m,
     }
     print(json.dumps(line), flush=True)
 
 
-def main():
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def torchrun_argv(argv, gpus, port):
+    """The command that re-runs this script with one process per GPU."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={gpus}",
+            "--master-addr=127.0.0.1", f"--master-port={port}", os.path.abspath(__file__)] + list(argv)
+
+
+def main(argv=None):
+    argv = sys.argv[1:] if argv is None else argv
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
@@ -438,13 +766,22 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-small-m", action="store_true")
-    args = ap.parse_args()
+    ap.add_argument("--block-only", action="store_true", help="only the headline block step")
+    args = ap.parse_args(argv)
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        # One process per GPU: re-launch under torch.distributed.run.
+        env = dict(os.environ)
+        env.setdefault("NCCL_DEBUG", "INFO")
+        env.setdefault("NCCL_DEBUG_SUBSYS", "INIT")
+        return subprocess.call(torchrun_argv(argv, args.gpus, _free_port()), env=env)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}: launch one process per GPU")
     if args.impl == "reference":
         run_reference(args, rank, world)
-        return
+        return 0
     if world > 1:
         import datetime
 
@@ -458,7 +795,8 @@ def main():
         if world > 1:
             import torch.distributed as dist
             dist.destroy_process_group()
+    return 0
 
 
 if __name__ == "__main__":
-    main()
+    sys.exit(main())

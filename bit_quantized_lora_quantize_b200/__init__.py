@@ -15,6 +15,8 @@ from .qlora import (  # noqa: F401
     qlora_check_status,
     qlora_get_wait_timeout,
     qlora_set_wait_timeout,
+    qlora_silu_gate_bwd,
+    qlora_silu_gate_fwd,
     qlora_dequantize_nf4,
     qlora_linear_bwd,
     qlora_linear_fwd,

@@ -249,6 +249,27 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float
   return QLORA_OK;
 }
 
+qlora_status qlora_silu_gate_fwd(const uint16_t* G, const uint16_t* U, uint16_t* H, int64_t n, void* stream) {
+  if (!G || !U || !H || n <= 0) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(G) || !aligned16(U) || !aligned16(H)) return QLORA_ERR_ALIGNMENT;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  ProfScope p(st, "silu_gate_fwd", 1);
+  const cudaError_t e = launch_silu_gate_fwd(G, U, H, n, st);
+  p.done();
+  return e == cudaSuccess ? QLORA_OK : cuda_fail(e);
+}
+
+qlora_status qlora_silu_gate_bwd(const uint16_t* G, const uint16_t* U, const uint16_t* dH, uint16_t* dG,
+                                 uint16_t* dU, int64_t n, void* stream) {
+  if (!G || !U || !dH || !dG || !dU || n <= 0) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(G) || !aligned16(U) || !aligned16(dH) || !aligned16(dG) || !aligned16(dU)) return QLORA_ERR_ALIGNMENT;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  ProfScope p(st, "silu_gate_bwd", 1);
+  const cudaError_t e = launch_silu_gate_bwd(G, U, dH, dG, dU, n, st);
+  p.done();
+  return e == cudaSuccess ? QLORA_OK : cuda_fail(e);
+}
+
 qlora_status qlora_check_status(void* workspace, void* stream) {
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaStreamSynchronize(st);

@@ -66,6 +66,8 @@ constexpr int kDecWarps = 4;      // decoder warps per stage (warps 4-7 even sta
 struct PairArgs {
   int units;        // CTA pairs in the grid
   int tiles_n;      // output tiles along the columns
+  int tiles_m;      // output tiles along the rows (512-row blocks)
+  int group_rows;   // row blocks per tile group (tile order, see tile_coords)
   // Rank units (one per 512-row block) ahead of the output tiles, or 0 when
   // the bf16 pair comes from the previous kernel in the stream.
   int r_units;
@@ -125,6 +127,23 @@ struct PairSmem {
   static constexpr int kTotal = offUnit + 4;
   static constexpr int kDynamic = kTotal + 1024;
 };
+
+// Output tile order.  Tiles go out in groups of `group_rows` consecutive
+// 512-row blocks; inside a group, column by column, each column's row blocks
+// in turn.  The activation rows of a group (group_rows x 512 x depth bf16)
+// are sized on the host to stay in L2 while the group sweeps its columns, and
+// the pairs working at the same time share the packed codes of a few
+// columns, so each code tile comes from HBM about once per group instead of
+// once per row block.
+__device__ __forceinline__ void tile_coords(int tile, int tiles_m, int tiles_n, int group_rows, int& tm, int& tn) {
+  const int per_group = group_rows * tiles_n;
+  const int g = tile / per_group;
+  const int idx = tile - g * per_group;
+  const int r0 = g * group_rows;
+  const int rows = min(group_rows, tiles_m - r0);
+  tn = idx / rows;
+  tm = r0 + (idx - tn * rows);
+}
 
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
@@ -266,8 +285,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     else tj = v - ntiles;
   }
   const bool tunit = tj >= 0;
-  const int tile_m = runit ? unit : tile / args.tiles_n;
-  const int tile_n = tile % args.tiles_n;
+  int tile_m = unit, tile_n = 0;
+  if (!runit) tile_coords(tile, args.tiles_m, args.tiles_n, args.group_rows, tile_m, tile_n);
   const int total = runit ? args.nkb : (tunit ? args.nmb : args.nkb + args.lora_kb);
   // Without rank units the previous kernel produces only the LoRA
   // intermediate, read in the last stages: everything else may start now.
@@ -748,12 +767,37 @@ cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& c, const CUtens
   return cudaLaunchKernelEx(&cfg, kern, a, c, a2, b2, abs, rmap, tmaps, args);
 }
 
-// Unit count and rank-unit fields shared by both directions.
-void plan_units(PairArgs& args, int64_t M, int64_t cols, int r, float scale, int* ctr, float* r_f32,
-                uint16_t* r_pair) {
+int l2_bytes() {
+  static int cached[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 126 << 20;
+  if (!cached[dev]) {
+    int v = 0;
+    cudaDeviceGetAttribute(&v, cudaDevAttrL2CacheSize, dev);
+    cached[dev] = v > 0 ? v : (126 << 20);
+  }
+  return cached[dev];
+}
+
+// Row blocks per tile group: as few groups as keep one group's activation
+// rows (512 x depth bf16 per row block) within half of L2, balanced.
+int group_rows_for(int tiles_m, int64_t depth) {
+  const int64_t block_bytes = static_cast<int64_t>(kPairRows) * depth * 2;
+  const int64_t budget = l2_bytes() / 2;
+  const int64_t fit = std::max<int64_t>(1, budget / std::max<int64_t>(1, block_bytes));
+  const int64_t groups = (tiles_m + fit - 1) / fit;
+  return static_cast<int>((tiles_m + groups - 1) / groups);
+}
+
+// Unit count and rank-unit fields shared by both directions.  `depth` is the
+// reduction length of the output tiles (K forward, N input gradient).
+void plan_units(PairArgs& args, int64_t M, int64_t cols, int64_t depth, int r, float scale, int* ctr,
+                float* r_f32, uint16_t* r_pair) {
   const int tiles_n = static_cast<int>((cols + kPairCols - 1) / kPairCols);
   const int tiles_m = static_cast<int>((M + kPairRows - 1) / kPairRows);
   args.tiles_n = tiles_n;
+  args.tiles_m = tiles_m;
+  args.group_rows = group_rows_for(tiles_m, depth);
   args.r_units = ctr ? tiles_m : 0;
   args.units = tiles_m * tiles_n + args.r_units;
   args.ctr = ctr;
@@ -797,7 +841,7 @@ cudaError_t launch_fused_fwd(const uint16_t* X, const uint8_t* codes, const uint
       return cudaErrorInvalidValue;
   }
   PairArgs args{};
-  plan_units(args, M, N, r, scale, ctr, T_save, Tpair);
+  plan_units(args, M, N, K, r, scale, ctr, T_save, Tpair);
   args.nkb = static_cast<int>(K / 64);
   args.lora_kb = 2 * rp / 64;
   args.lora_mod = rp;
@@ -842,7 +886,7 @@ cudaError_t launch_fused_dx(const uint16_t* dY, const uint8_t* codes, const uint
                        make_map_2d(&mAbs, CU_TENSOR_MAP_DATA_TYPE_UINT8, absmax_q, K / 64, N, K / 64, 16, 64,
                                    CU_TENSOR_MAP_SWIZZLE_NONE);
   PairArgs args{};
-  plan_units(args, M, K, r, scale, ctr, nullptr, Upair);
+  plan_units(args, M, K, N, r, scale, ctr, nullptr, Upair);
   TailMaps tails{mA, mA, mA, mA};
   if (ctr && dA && dB) {
     // dA = X^T U and dB^T = dY^T T: 64 tokens x 64 result rows per box

@@ -82,4 +82,10 @@ cudaError_t launch_small_m_fwd(const uint16_t* X, const uint8_t* codes, const ui
                                int64_t K, int64_t N, int r, float scale, uint16_t* Y, float* T_save, uint16_t* Tpair,
                                void* scratch, int* status, const Nf4Params& P, cudaStream_t stream);
 
+// SiLU gate of a gated MLP (glue between linears): H = silu(G) * U and its
+// backward dG, dU, elementwise over n bf16 values.
+cudaError_t launch_silu_gate_fwd(const uint16_t* G, const uint16_t* U, uint16_t* H, int64_t n, cudaStream_t stream);
+cudaError_t launch_silu_gate_bwd(const uint16_t* G, const uint16_t* U, const uint16_t* dH, uint16_t* dG,
+                                 uint16_t* dU, int64_t n, cudaStream_t stream);
+
 }  // namespace qlora

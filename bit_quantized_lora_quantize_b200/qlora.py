@@ -33,6 +33,8 @@ _SIGS = {
                                         ctypes.c_float, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "qlora_linear_fwd_noalloc": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, ctypes.c_int32,
                                                 ctypes.c_float, _P, _P, _P]),
+    "qlora_silu_gate_fwd": (ctypes.c_int, [_P, _P, _P, _I64, _P]),
+    "qlora_silu_gate_bwd": (ctypes.c_int, [_P, _P, _P, _P, _P, _I64, _P]),
     "qlora_workspace_bytes": (ctypes.c_size_t, [_I64, _I64, _I64, ctypes.c_int32]),
     "qlora_check_status": (ctypes.c_int, [_P, _P]),
     "qlora_set_wait_timeout": (ctypes.c_int, [ctypes.c_uint64]),
@@ -228,6 +230,33 @@ def qlora_linear_bwd(dY: torch.Tensor, X: torch.Tensor, T_save: torch.Tensor, W:
     return dX, dA, dB
 
 
+def _same_bf16(*ts: torch.Tensor) -> None:
+    _require_cuda(*ts)
+    for t in ts:
+        if t.dtype != torch.bfloat16 or t.numel() != ts[0].numel():
+            raise ValueError("bf16 tensors of one size expected")
+
+
+def qlora_silu_gate_fwd(G: torch.Tensor, U: torch.Tensor, H: torch.Tensor | None = None) -> torch.Tensor:
+    """H = silu(G) * U (glue between the linears of a gated MLP)."""
+    if H is None:
+        H = torch.empty_like(G)
+    _same_bf16(G, U, H)
+    _check("qlora_silu_gate_fwd", lib().qlora_silu_gate_fwd(_ptr(G), _ptr(U), _ptr(H), G.numel(), _stream()))
+    return H
+
+
+def qlora_silu_gate_bwd(G: torch.Tensor, U: torch.Tensor, dH: torch.Tensor, dG: torch.Tensor | None = None,
+                        dU: torch.Tensor | None = None):
+    """(dG, dU) of H = silu(G) * U for the upstream gradient dH."""
+    dG = torch.empty_like(G) if dG is None else dG
+    dU = torch.empty_like(U) if dU is None else dU
+    _same_bf16(G, U, dH, dG, dU)
+    _check("qlora_silu_gate_bwd", lib().qlora_silu_gate_bwd(_ptr(G), _ptr(U), _ptr(dH), _ptr(dG), _ptr(dU),
+                                                            G.numel(), _stream()))
+    return dG, dU
+
+
 def qlora_check_status(workspace: torch.Tensor | None = None) -> int:
     """Synchronise and return the device status code (0 = OK, 6 = a pipeline
     wait timed out): the workspace's word (if given) and the library's own
@@ -265,4 +294,5 @@ def qlora_profile_stop(max_entries: int = 32) -> dict:
 __all__ = ["qlora_profile_start", "qlora_profile_stop", "LIB_PATH", "lib", "QloraError", "PackedNF4", "packed_sizes", "qlora_nf4_codebook", "qlora_quantize_nf4",
            "qlora_dequantize_nf4", "qlora_workspace_bytes", "new_workspace", "qlora_linear_fwd", "qlora_linear_bwd",
            "qlora_linear_fwd_noalloc",
-           "qlora_check_status", "qlora_set_wait_timeout", "qlora_get_wait_timeout"]
+           "qlora_check_status", "qlora_set_wait_timeout", "qlora_get_wait_timeout", "qlora_silu_gate_fwd",
+           "qlora_silu_gate_bwd"]

@@ -124,5 +124,68 @@ def small_m_case(M: int, N: int, K: int = 8192, seed: int = 4) -> LinearCase:
     return linear_case(M, K, N, 64, 0.25, seed, with_dy=False)
 
 
+# The seven linears of a LLaMA-65B-shaped block: (name, out N, in K).
+LLAMA65B_LINEARS = (("q", 8192, 8192), ("k", 8192, 8192), ("v", 8192, 8192), ("o", 8192, 8192),
+                    ("gate", 22016, 8192), ("up", 22016, 8192), ("down", 8192, 22016))
+
+
+def llama65b_block(M: int = 4096, r: int = 64, scale: float = 0.25) -> list:
+    """LLaMA-65B-shaped block linears, M tokens (seed family 3).
+
+    Weight i is the 'W' stream of seed 300 + i (the same weights the one-shot
+    quantization test uses); the six linears with in-dim 8192 share one input
+    X (the 'X' stream of seed 3); the down projection takes its own
+    M x 22016 input (the 'extra0' stream of seed 3).  Adapter i and its dY
+    come from the A, B and dY streams of seed 310 + i.  Returns a list of
+    (name, LinearCase)."""
+    st = Streams(3)
+    X = to_bf16(normal(st["X"], (M, 8192), 1.0))
+    Xd = to_bf16(normal(st["extra0"], (M, 22016), 1.0))
+    out = []
+    for i, (name, N, K) in enumerate(LLAMA65B_LINEARS):
+        w = weight_only(N, K, seed=300 + i)
+        sa = Streams(310 + i)
+        a = to_bf16(normal(sa["A"], (K, r), 0.01))
+        b = to_bf16(normal(sa["B"], (r, N), 0.01))
+        dy = to_bf16(normal(sa["dY"], (M, N), 1.0))
+        out.append((name, LinearCase(W=w, X=X if K == 8192 else Xd, A=a, B=b, dY=dy, scale=float(scale),
+                                     meta=dict(seed=300 + i))))
+    return out
+
+
+@dataclass
+class MlpTrio:
+    """LLaMA-7B MLP: gate/up [F x D], down [D x F], X [M x D], dY [M x D]."""
+
+    Wg: torch.Tensor
+    Wu: torch.Tensor
+    Wd: torch.Tensor
+    X: torch.Tensor
+    Ag: torch.Tensor
+    Au: torch.Tensor
+    Ad: torch.Tensor
+    Bg: torch.Tensor
+    Bu: torch.Tensor
+    Bd: torch.Tensor
+    dY: torch.Tensor
+    scale: float
+
+
+def mlp_trio(M: int = 8192, D: int = 4096, F: int = 11008, r: int = 64, scale: float = 0.25) -> MlpTrio:
+    """LLaMA-7B MLP trio inputs (seed 2), drawn in a fixed stream order."""
+    st = Streams(2)
+    Wg = to_bf16(normal(st["W"], (F, D), 0.02))
+    Wu = to_bf16(normal(st["outliers"], (F, D), 0.02))
+    Wd = to_bf16(normal(st["extra0"], (D, F), 0.02))
+    X = to_bf16(normal(st["X"], (M, D), 1.0))
+    Ag, Au = (to_bf16(normal(st["A"], (D, r), 0.01)) for _ in range(2))
+    Ad = to_bf16(normal(st["A"], (F, r), 0.01))
+    Bg, Bu = (to_bf16(normal(st["B"], (r, F), 0.01)) for _ in range(2))
+    Bd = to_bf16(normal(st["B"], (r, D), 0.01))
+    dY = to_bf16(normal(st["dY"], (M, D), 1.0))
+    return MlpTrio(Wg, Wu, Wd, X, Ag, Au, Ad, Bg, Bu, Bd, dY, float(scale))
+
+
 __all__ = ["to_bf16", "Streams", "LinearCase", "linear_case", "weight_only",
-           "tiny_case", "attn_proj_case", "small_m_case"]
+           "tiny_case", "attn_proj_case", "small_m_case", "LLAMA65B_LINEARS", "llama65b_block",
+           "MlpTrio", "mlp_trio"]

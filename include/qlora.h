@@ -196,6 +196,21 @@ QLORA_API qlora_status qlora_linear_fwd_noalloc(const uint16_t* X, int64_t M, in
                                                 const float* absmax_scale, const uint16_t* A, const uint16_t* B,
                                                 int32_t r, float scale, uint16_t* Y, float* T_save, void* stream);
 
+/*
+ * SiLU gate between the linears of a gated MLP (the LLaMA feed-forward block
+ * the QLoRA experiments fine-tune): glue between LoRA linears, not a step of
+ * the method, so the pages have no counterpart.  Elementwise over n values,
+ * float32 arithmetic, one bf16 rounding per output:
+ *   forward   H  = silu(G) * U = G * sigmoid(G) * U
+ *   backward  dG = dH * U * sigmoid(G) * (1 + G * (1 - sigmoid(G)))
+ *             dU = dH * G * sigmoid(G)
+ * All pointers bf16[n], 16-byte aligned; outputs may not alias inputs.
+ */
+QLORA_API qlora_status qlora_silu_gate_fwd(const uint16_t* G, const uint16_t* U, uint16_t* H, int64_t n,
+                                           void* stream);
+QLORA_API qlora_status qlora_silu_gate_bwd(const uint16_t* G, const uint16_t* U, const uint16_t* dH, uint16_t* dG,
+                                           uint16_t* dU, int64_t n, void* stream);
+
 /* Workspace bytes needed by qlora_linear_fwd / qlora_linear_bwd for these sizes
  * (0 for an unsupported shape). */
 QLORA_API size_t qlora_workspace_bytes(int64_t M, int64_t K, int64_t N, int32_t r);

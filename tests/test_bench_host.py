@@ -1,7 +1,8 @@
 """Host-side logic of bench.py that needs no GPU: the clock sampler (run
 against a fake NVML module in the child process it starts), the rule that
 keeps a committed DRAM-traffic figure only while its kernel's sources are
-unchanged, and the oracle reference arm's JSON line."""
+unchanged, the oracle reference arm's JSON line, and the multi-GPU launch
+(re-execution under torchrun, world-size check)."""
 import sys
 import time
 
@@ -95,4 +96,27 @@ def test_reference_arm_prints_the_contract_line():
     assert d["value"] > 0 and d["ms_per_step"] > 0 and d["tokens_per_s"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"] == {"value": d["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
-    assert d["config"]["workload"] == "llama7b_attn_proj_qlora_linear"
+    assert d["config"]["workload"] == "llama65b_block_linears"
+    import os
+    assert d["cpu_baseline"]["cores"] == len(os.sched_getaffinity(0))
+
+
+def test_multi_gpu_launch_re_execs_under_torchrun():
+    """`bench.py --gpus N` without torchrun re-launches itself with one
+    process per GPU; under torchrun a world size other than N is an error."""
+    import bench
+
+    cmd = bench.torchrun_argv(["--gpus", "2", "--steps", "3"], 2, 29511)
+    assert cmd[1:3] == ["-m", "torch.distributed.run"]
+    assert "--nproc-per-node=2" in cmd and "--master-addr=127.0.0.1" in cmd and "--master-port=29511" in cmd
+    assert cmd[-3:] == ["--gpus", "2", "--steps", "3"][-3:] and cmd[-4] == "--gpus"
+    assert cmd.index(bench.__file__.replace(".pyc", ".py")) < cmd.index("--gpus")
+
+
+def test_world_size_must_match_gpus(monkeypatch):
+    import bench
+
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    monkeypatch.setenv("RANK", "0")
+    with pytest.raises(SystemExit):
+        bench.main(["--gpus", "4"])

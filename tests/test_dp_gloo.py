@@ -1,6 +1,8 @@
 """Data-parallel exchange on CPU: two gloo ranks each take their share of the
-tokens, compute the adapter gradients with the oracle, sum them with the
-reducer the benchmark uses, and must reproduce the full-batch gradients."""
+tokens, compute the adapter gradients of two linears with the oracle into
+views of one gradient bucket (the structure the benchmark's backward writes
+into), sum the bucket with its all-reduce, and must reproduce the full-batch
+gradients."""
 
 import os
 import socket
@@ -30,21 +32,35 @@ def _rank_main(rank, world, port, out):
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
-        case = synthetic.linear_case(37, 128, 96, 8, 0.5, seed=77)
-        codes, aq, sc = quantize_nf4(case.W.float().numpy())
-        Wdq = dequantize_nf4(codes, aq, sc, case.W.numel()).reshape(case.N, case.K)
-        rows = dp.shard_rows(case.M, rank, world)
-        X = case.X[rows].double().numpy()
-        dY = case.dY[rows].double().numpy()
-        _, dA, dB = lora_linear_backward(dY, X, Wdq, case.A.double().numpy(), case.B.double().numpy(), case.scale)
-        tA = torch.from_numpy(dA.astype(np.float32))
-        tB = torch.from_numpy(dB.astype(np.float32))
-        dp.AdapterGradReducer(case.K, case.N, case.r, "cpu")(tA, tB)
+        # Two linears of different shapes share one bucket, as the block
+        # step's seven linears do.
+        cases = [synthetic.linear_case(37, 128, 96, 8, 0.5, seed=77),
+                 synthetic.linear_case(37, 64, 200, 16, 0.25, seed=78)]
+        bucket = dp.GradBucket([(c.K, c.N, c.r) for c in cases], "cpu")
+        rows = dp.shard_rows(cases[0].M, rank, world)
+        fulls = []
+        for i, case in enumerate(cases):
+            codes, aq, sc = quantize_nf4(case.W.float().numpy())
+            Wdq = dequantize_nf4(codes, aq, sc, case.W.numel()).reshape(case.N, case.K)
+            X = case.X[rows].double().numpy()
+            dY = case.dY[rows].double().numpy()
+            A, B = case.A.double().numpy(), case.B.double().numpy()
+            _, dA, dB = lora_linear_backward(dY, X, Wdq, A, B, case.scale)
+            vA, vB = bucket[i]
+            vA.copy_(torch.from_numpy(dA.astype(np.float32)))
+            vB.copy_(torch.from_numpy(dB.astype(np.float32)))
+            if rank == 0:
+                _, fA, fB = lora_linear_backward(case.dY.double().numpy(), case.X.double().numpy(), Wdq, A, B,
+                                                 case.scale)
+                fulls.append((fA, fB))
+        bucket.all_reduce()
         if rank == 0:
-            _, fA, fB = lora_linear_backward(case.dY.double().numpy(), case.X.double().numpy(), Wdq,
-                                             case.A.double().numpy(), case.B.double().numpy(), case.scale)
-            out["errA"] = float(np.max(np.abs(tA.numpy() - fA)) / np.sqrt(np.mean(fA ** 2)))
-            out["errB"] = float(np.max(np.abs(tB.numpy() - fB)) / np.sqrt(np.mean(fB ** 2)))
+            errs = []
+            for i, (fA, fB) in enumerate(fulls):
+                vA, vB = bucket[i]
+                errs.append(float(np.max(np.abs(vA.numpy() - fA)) / np.sqrt(np.mean(fA ** 2))))
+                errs.append(float(np.max(np.abs(vB.numpy() - fB)) / np.sqrt(np.mean(fB ** 2))))
+            out["errs"] = errs
     finally:
         dist.destroy_process_group()
 
@@ -64,4 +80,4 @@ def test_two_rank_gradient_sum_equals_full_batch():
     with mp.Manager() as m:
         out = m.dict()
         mp.spawn(_rank_main, args=(2, port, out), nprocs=2, join=True)
-        assert out["errA"] < 1e-5 and out["errB"] < 1e-5
+        assert len(out["errs"]) == 4 and max(out["errs"]) < 1e-5, out["errs"]

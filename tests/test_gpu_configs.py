@@ -108,35 +108,27 @@ def test_mlp_trio_linear_shapes(name, K, N):
 def test_mlp_trio_chain():
     """Y = down(silu(gate(X)) * up(X)) and its input gradient, on sampled rows.
 
-    The SiLU gate is harness glue (torch, float32 -> bf16) between the three
-    LoRA linears; every linear runs through the library."""
-    st = synthetic.Streams(2)
-    M, D, F, r, s = 8192, 4096, 11008, 64, 0.25
-    Wg = synthetic.to_bf16(synthetic.normal(st["W"], (F, D), 0.02))
-    Wu = synthetic.to_bf16(synthetic.normal(st["outliers"], (F, D), 0.02))
-    Wd = synthetic.to_bf16(synthetic.normal(st["extra0"], (D, F), 0.02))
-    X = synthetic.to_bf16(synthetic.normal(st["X"], (M, D), 1.0))
-    Ag, Au = (synthetic.to_bf16(synthetic.normal(st["A"], (D, r), 0.01)) for _ in range(2))
-    Ad = synthetic.to_bf16(synthetic.normal(st["A"], (F, r), 0.01))
-    Bg, Bu = (synthetic.to_bf16(synthetic.normal(st["B"], (r, F), 0.01)) for _ in range(2))
-    Bd = synthetic.to_bf16(synthetic.normal(st["B"], (r, D), 0.01))
-    dY = synthetic.to_bf16(synthetic.normal(st["dY"], (M, D), 1.0))
+    The SiLU gate is glue between the three LoRA linears (the library's
+    elementwise kernels, float32 arithmetic, bf16 outputs); every linear runs
+    through the library."""
+    M, D, F, r = 8192, 4096, 11008, 64
+    t = synthetic.mlp_trio(M, D, F, r, 0.25)
+    s = t.scale
+    Wg, Wu, Wd, X, dY = t.Wg, t.Wu, t.Wd, t.X, t.dY
+    Ag, Au, Ad, Bg, Bu, Bd = t.Ag, t.Au, t.Ad, t.Bg, t.Bu, t.Bd
 
     d = lambda t: t.to(DEV)  # noqa: E731
     Pg, Pu, Pd = (q.qlora_quantize_nf4(d(w)) for w in (Wg, Wu, Wd))
     G, Tg = q.qlora_linear_fwd(d(X), Pg, d(Ag), d(Bg), s)
     Up, Tu = q.qlora_linear_fwd(d(X), Pu, d(Au), d(Bu), s)
-    Gf, Uf = G.float(), Up.float()
-    H = (torch.nn.functional.silu(Gf) * Uf).to(torch.bfloat16)
+    H = q.qlora_silu_gate_fwd(G, Up)
     Y, Td = q.qlora_linear_fwd(H, Pd, d(Ad), d(Bd), s)
     dH, _, _ = q.qlora_linear_bwd(d(dY), H, Td, Pd, d(Ad), d(Bd), s)
-    sg = torch.sigmoid(Gf)
-    dHf = dH.float()
-    dG = (dHf * Uf * sg * (1 + Gf * (1 - sg))).to(torch.bfloat16)
-    dU = (dHf * Gf * sg).to(torch.bfloat16)
+    dG, dU = q.qlora_silu_gate_bwd(G, Up, dH)
     dXg, _, _ = q.qlora_linear_bwd(dG, d(X), Tg, Pg, d(Ag), d(Bg), s)
     dXu, _, _ = q.qlora_linear_bwd(dU, d(X), Tu, Pu, d(Au), d(Bu), s)
     dX = dXg.float() + dXu.float()
+    assert q.qlora_check_status(None) == 0
 
     rows = sample(M, 32, 11)
     Xr = f64(X)[rows]
