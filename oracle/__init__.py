@@ -21,6 +21,10 @@ Parity status per function (see each module's header):
                             normal-quantile routes, equal-probability spacing);
                             the numeric values themselves are not printed on
                             the pages.
+  * fp4/int4_codebook       pinned to the reading (the printed rationals of
+                            the 1-2-1 float and k/7, invariants) and to the
+                            pages' claim that NF4 has the lower error on
+                            normally distributed weights.
   * quantize / dequantize   pinned (brute force on tiny inputs in exact
                             rational arithmetic, closed forms, special cases).
   * forward / backward      pinned (finite differences, torch fp64 autograd,
@@ -31,6 +35,9 @@ from .nf4_ref import (  # noqa: F401
     BLOCK,
     GROUP,
     nf4_codebook,
+    fp4_codebook,
+    int4_codebook,
+    codebook,
     bf16_round,
     quantize_nf4,
     dequantize_nf4,

@@ -31,6 +31,20 @@ What the pages fix, and the readings taken where they are silent:
   used.  Reading: a' = fp32(fp32(k/255) * c1); w' = bf16(fp32(q_code * a')),
   each product a single correctly rounded float32 multiply, bf16 by
   round-to-nearest-even.
+* "1. 4-bit NormalFloat (NF4)" names the usual 4-bit alternatives, Integer
+  4-bit and Float 4-bit, and claims NF4 has the lower quantization error
+  ("Performance and Evaluation", "NF4 efficiency"; the glossary's third
+  paragraph: a plain 4-bit float scored about a point lower).  Neither format
+  is defined on the pages.  Readings, both with the same block scaling,
+  packing and double quantization as NF4, so only the 16 levels change:
+    FP4  the 4-bit float with 1 sign, 2 exponent and 1 mantissa bit (bias 1,
+         subnormals at exponent 0): magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6,
+         divided by the largest, 6, so that the block absmax maps to +-1;
+    Int4 the symmetric absmax integer code k/7, k = -7 .. 7.
+  Each has 15 distinct values (FP4's +0 and -0 coincide); sorted, they fill
+  indices 0..14 with the zero at index 7, and index 15 repeats the top level
+  +1.  Ties go to the lower index, so code 15 is never produced and every
+  code's value is the index's level, as for NF4.
 """
 
 from __future__ import annotations
@@ -61,6 +75,33 @@ def nf4_codebook() -> np.ndarray:
     levels = np.array(sorted(pos + neg + [0.0]), dtype=np.float64)
     levels = levels / levels.max()
     return levels.astype(np.float32)
+
+
+def fp4_codebook() -> np.ndarray:
+    """The FP4 (1-2-1 float) levels as float32, sorted, divided by 6; index
+    15 repeats +1 (see the module header)."""
+    mags = []
+    for m in range(8):  # 2 exponent bits, 1 mantissa bit
+        e, f = m >> 1, m & 1
+        mags.append(f * 0.5 if e == 0 else (1.0 + 0.5 * f) * 2.0 ** (e - 1))
+    vals = sorted({v * sgn for v in mags for sgn in (1.0, -1.0)})  # 15 distinct (+-0 coincide)
+    vals = np.array(vals + [max(vals)], dtype=np.float64) / max(mags)
+    return vals.astype(np.float32)
+
+
+def int4_codebook() -> np.ndarray:
+    """The symmetric Int4 levels k/7, k = -7..7, as float32; index 15
+    repeats +1 (see the module header)."""
+    k = np.concatenate([np.arange(-7, 8), [7]]).astype(np.float64)
+    return (k / 7.0).astype(np.float32)
+
+
+CODEBOOKS = {"nf4": nf4_codebook, "fp4": fp4_codebook, "int4": int4_codebook}
+
+
+def codebook(name: str = "nf4") -> np.ndarray:
+    """The 16 float32 levels of the named 4-bit code ("nf4", "fp4", "int4")."""
+    return CODEBOOKS[name]()
 
 
 def bf16_round(x: np.ndarray) -> np.ndarray:
@@ -98,8 +139,9 @@ def _level2_table() -> np.ndarray:
     return (np.arange(256, dtype=np.float64) / 255.0).astype(np.float32)
 
 
-def quantize_nf4(w: np.ndarray, block: int = BLOCK, group: int = GROUP):
-    """Blockwise NF4 quantization with double-quantized constants.
+def quantize_nf4(w: np.ndarray, block: int = BLOCK, group: int = GROUP, code: str = "nf4"):
+    """Blockwise NF4 quantization with double-quantized constants (or the
+    same scheme with the FP4 or Int4 levels, ``code`` = "fp4" / "int4").
 
     ``w``: any-shape array of bfloat16 values (given as float32/float64 that
     lie on the bf16 grid), flattened row-major.
@@ -118,7 +160,7 @@ def quantize_nf4(w: np.ndarray, block: int = BLOCK, group: int = GROUP):
     x = np.asarray(w, dtype=np.float32).reshape(-1)
     n = x.size
     nb = -(-n // block)
-    q = nf4_codebook()
+    q = codebook(code)
 
     # Level 1: per-block absmax c_b over the elements present.
     padded = np.zeros(nb * block, dtype=np.float32)
@@ -167,7 +209,7 @@ def dequantize_scales(absmax_q: np.ndarray, absmax_scale: np.ndarray, group: int
 
 
 def dequantize_nf4(codes: np.ndarray, absmax_q: np.ndarray, absmax_scale: np.ndarray,
-                   numel: int, block: int = BLOCK, group: int = GROUP) -> np.ndarray:
+                   numel: int, block: int = BLOCK, group: int = GROUP, code: str = "nf4") -> np.ndarray:
     """Dequantize to bfloat16 values (returned as float32 on the bf16 grid).
 
     w' = bf16(fp32(q_code * a')), a' from :func:`dequantize_scales`.
@@ -177,14 +219,15 @@ def dequantize_nf4(codes: np.ndarray, absmax_q: np.ndarray, absmax_scale: np.nda
     nib[0::2] = packed >> 4
     nib[1::2] = packed & 0xF
     nib = nib[:numel]
-    q = nf4_codebook().astype(np.float64)
+    q = codebook(code).astype(np.float64)
     a = dequantize_scales(absmax_q, absmax_scale, group)
     ab = np.repeat(a, block)[:numel].astype(np.float64)
     w32 = (q[nib] * ab).astype(np.float32)  # exact float64 product, one rounding
     return bf16_round(w32)
 
 
-def dequantize_at(w: np.ndarray, flat_idx: np.ndarray, block: int = BLOCK, group: int = GROUP) -> np.ndarray:
+def dequantize_at(w: np.ndarray, flat_idx: np.ndarray, block: int = BLOCK, group: int = GROUP,
+                  code: str = "nf4") -> np.ndarray:
     """Quantize-then-dequantize only the elements at ``flat_idx`` of ``w``.
 
     Same definitions as :func:`quantize_nf4` followed by
@@ -210,15 +253,15 @@ def dequantize_at(w: np.ndarray, flat_idx: np.ndarray, block: int = BLOCK, group
     with np.errstate(invalid="ignore", divide="ignore"):
         normed = (x[idx].astype(np.float64) / cb.astype(np.float64)).astype(np.float32)
     normed = np.where(cb == 0, np.float32(0.0), normed)
-    q = nf4_codebook()
-    code = _nearest_index(normed, q)
+    q = codebook(code)
+    idx_code = _nearest_index(normed, q)
     c1b = c1[b // group]
     with np.errstate(invalid="ignore", divide="ignore"):
         n2 = (cb.astype(np.float64) / c1b.astype(np.float64)).astype(np.float32)
     n2 = np.where(c1b == 0, np.float32(0.0), n2)
     code2 = _nearest_index(n2, _level2_table())
     a = (_level2_table()[code2].astype(np.float64) * c1b.astype(np.float64)).astype(np.float32)
-    w32 = (q.astype(np.float64)[code] * a.astype(np.float64)).astype(np.float32)
+    w32 = (q.astype(np.float64)[idx_code] * a.astype(np.float64)).astype(np.float32)
     return bf16_round(w32)
 
 
@@ -229,14 +272,15 @@ def bits_per_parameter(numel: int, block: int = BLOCK, group: int = GROUP) -> fl
     return (8.0 * ((numel + 1) // 2) + 8.0 * nb + 32.0 * nb2) / numel
 
 
-def max_half_gap() -> float:
-    """Largest distance from a value in [-1, 1] to its nearest NF4 level."""
-    q = nf4_codebook().astype(np.float64)
+def max_half_gap(code: str = "nf4") -> float:
+    """Largest distance from a value in [-1, 1] to its nearest level."""
+    q = codebook(code).astype(np.float64)
     return float(np.max(np.diff(q)) / 2.0)
 
 
 __all__ = [
-    "BLOCK", "GROUP", "ZERO_CODE", "nf4_codebook", "bf16_round", "bf16_bits",
+    "BLOCK", "GROUP", "ZERO_CODE", "nf4_codebook", "fp4_codebook", "int4_codebook", "CODEBOOKS", "codebook",
+    "bf16_round", "bf16_bits",
     "quantize_nf4", "dequantize_scales", "dequantize_nf4", "dequantize_at", "bits_per_parameter",
     "max_half_gap",
 ]

@@ -24,6 +24,15 @@ from tests.exact import frac, rn_f32, rn_bf16
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 Q = [frac(v) for v in nf4_codebook()]
 L2 = [rn_f32(Fraction(k, 255)) for k in range(256)]
+# The FP4 and Int4 readings written out as rationals (see
+# tests/test_oracle_codebook.py), rounded to float32 exactly.
+_FP4_POS = [Fraction(1, 12), Fraction(1, 6), Fraction(1, 4), Fraction(1, 3), Fraction(1, 2), Fraction(2, 3),
+            Fraction(1)]
+LEVELS = {
+    "nf4": Q,
+    "fp4": [rn_f32(v) for v in [-v for v in reversed(_FP4_POS)] + [Fraction(0)] + _FP4_POS + [Fraction(1)]],
+    "int4": [rn_f32(Fraction(k, 7)) for k in list(range(-7, 8)) + [7]],
+}
 
 
 def nearest(value, levels):
@@ -35,8 +44,9 @@ def nearest(value, levels):
     return best
 
 
-def brute_quantize(x, block=64, group=256):
+def brute_quantize(x, block=64, group=256, levels=None):
     """Element-by-element restatement of the codec (exact rationals)."""
+    levels = Q if levels is None else levels
     xs = [frac(v) for v in x]
     n = len(xs)
     nb = -(-n // block)
@@ -44,7 +54,7 @@ def brute_quantize(x, block=64, group=256):
     codes = []
     for i, v in enumerate(xs):
         cb = c[i // block]
-        codes.append(7 if cb == 0 else nearest(rn_f32(v / cb), Q))
+        codes.append(7 if cb == 0 else nearest(rn_f32(v / cb), levels))
     if n % 2:
         codes.append(7)
     packed = [codes[2 * j] * 16 + codes[2 * j + 1] for j in range(len(codes) // 2)]
@@ -57,7 +67,8 @@ def brute_quantize(x, block=64, group=256):
     return packed, code2, c1
 
 
-def brute_dequantize(packed, code2, c1, n, block=64, group=256):
+def brute_dequantize(packed, code2, c1, n, block=64, group=256, levels=None):
+    levels = Q if levels is None else levels
     nib = []
     for byte in packed:
         nib += [byte >> 4, byte & 15]
@@ -65,7 +76,7 @@ def brute_dequantize(packed, code2, c1, n, block=64, group=256):
     for i in range(n):
         b = i // block
         a = rn_f32(L2[code2[b]] * c1[b // group])
-        out.append(rn_bf16(rn_f32(Q[nib[i]] * a)))
+        out.append(rn_bf16(rn_f32(levels[nib[i]] * a)))
     return out
 
 
@@ -73,49 +84,55 @@ def bf16_values(rng, n, std):
     return bf16_round(rng.standard_normal(n).astype(np.float32) * np.float32(std))
 
 
+@pytest.mark.parametrize("code", ["nf4", "fp4", "int4"])
 @pytest.mark.parametrize("n", [1, 2, 63, 64, 65, 127, 130, 64 * 256 + 5])
-def test_quantize_matches_brute_force(n):
+def test_quantize_matches_brute_force(n, code):
+    if code != "nf4" and n not in (1, 65, 64 * 256 + 5):
+        pytest.skip("the other codebooks on a subset of the sizes")
     rng = np.random.default_rng(100 + n)
     x = bf16_values(rng, n, 0.02)
     if n > 70:
         x[64:128] = 0.0  # an all-zero block
-    packed, code2, c1 = quantize_nf4(x)
-    bp, bc2, bc1 = brute_quantize(list(x))
+    packed, code2, c1 = quantize_nf4(x, code=code)
+    bp, bc2, bc1 = brute_quantize(list(x), levels=LEVELS[code])
     assert packed.tolist() == bp
     assert code2.tolist() == bc2
     assert [frac(v) for v in c1] == bc1
 
 
-def test_dequantize_matches_brute_force():
+@pytest.mark.parametrize("code", ["nf4", "fp4", "int4"])
+def test_dequantize_matches_brute_force(code):
     rng = np.random.default_rng(7)
     n = 64 * 256 + 37
     x = bf16_values(rng, n, 0.05)
-    packed, code2, c1 = quantize_nf4(x)
-    got = dequantize_nf4(packed, code2, c1, n)
-    ref = brute_dequantize(packed.tolist(), code2.tolist(), [frac(v) for v in c1], n)
+    packed, code2, c1 = quantize_nf4(x, code=code)
+    got = dequantize_nf4(packed, code2, c1, n, code=code)
+    ref = brute_dequantize(packed.tolist(), code2.tolist(), [frac(v) for v in c1], n, levels=LEVELS[code])
     assert [frac(v) for v in got] == ref
 
 
-def test_every_bf16_pattern_against_exact_threshold():
+@pytest.mark.parametrize("code", ["nf4", "fp4", "int4"])
+def test_every_bf16_pattern_against_exact_threshold(code):
     """All finite bf16 values x with |x| <= c, for several block maxima c
     (including ones whose quotient x/c is not a float32, so the rounding of
     the scaled value matters), against exact midpoint counting."""
     bits = np.arange(65536, dtype=np.uint32) << 16
     allv = bits.view(np.float32)
     allv = allv[np.isfinite(allv)]
-    mids = [(Q[i] + Q[i + 1]) / 2 for i in range(15)]
-    for c in (1.0, 0.75, 0.0234375, 3.0):
+    lv = LEVELS[code]
+    mids = [(lv[i] + lv[i + 1]) / 2 for i in range(15)]
+    for c in ((1.0, 0.75, 0.0234375, 3.0) if code == "nf4" else (0.75, 3.0)):
         xs = allv[np.abs(allv) <= c]
         # Blocks of 64: [c, x, x, ..., x] so the block absmax is exactly c.
         blocks = np.repeat(xs[:, None], 64, axis=1)
         blocks[:, 0] = c
-        packed, _, _ = quantize_nf4(blocks.reshape(-1))
+        packed, _, _ = quantize_nf4(blocks.reshape(-1), code=code)
         codes = (packed.reshape(-1, 32)[:, 0] & 15)  # element 1 of each block
         cf = Fraction(c)
-        for x, code in zip(xs.tolist(), codes.tolist()):
+        for x, got in zip(xs.tolist(), codes.tolist()):
             nq = rn_f32(Fraction(x) / cf)
             ref = sum(1 for m in mids if nq > m)  # ties -> lower index
-            assert code == ref, (c, x, code, ref)
+            assert got == ref, (c, x, got, ref)
 
 
 def test_special_cases():
