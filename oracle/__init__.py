@@ -14,7 +14,7 @@ Sources (the pages describe the method in prose only):
   * "QLoRA: Fine-Tuning 65-Billion Parameter Models on a Single Consumer GPU"
     (deepfa.ir), sections "LoRA: Prerequisite for Understanding QLoRA",
     "QLoRA's Technical Innovations" (1. 4-bit NormalFloat, 2. Double
-    Quantization) and "QLoRA's Working Process".
+    Quantization, 3. Paged Optimizers) and "QLoRA's Working Process".
 
 Parity status per function (see each module's header):
   * nf4_codebook            pinned to the reading (invariants, two independent
@@ -29,6 +29,8 @@ Parity status per function (see each module's header):
                             rational arithmetic, closed forms, special cases).
   * forward / backward      pinned (finite differences, torch fp64 autograd,
                             special cases).
+  * adamw_step / adamw_run  pinned (closed forms of the first step and of a
+                            constant gradient, torch.optim.AdamW in float64).
 """
 
 from .nf4_ref import (  # noqa: F401
@@ -45,3 +47,4 @@ from .nf4_ref import (  # noqa: F401
     dequantize_at,
 )
 from .linear_ref import lora_linear_forward, lora_linear_backward  # noqa: F401
+from .adamw_ref import adamw_step, adamw_run  # noqa: F401
