@@ -145,30 +145,44 @@ using namespace qlora;
 
 extern "C" {
 
-qlora_status qlora_quantize_nf4(const uint16_t* W, int64_t numel, uint8_t* codes, uint8_t* absmax_q,
-                                float* absmax_scale, void* stream) {
+qlora_status qlora_quantize_4bit(const uint16_t* W, int64_t numel, int32_t code, uint8_t* codes, uint8_t* absmax_q,
+                                 float* absmax_scale, void* stream) {
   if (!W || !codes || !absmax_q || !absmax_scale || numel <= 0) return QLORA_ERR_INVALID_ARG;
+  const Nf4Params* P = code_params_or_null(code);
+  if (!P) return QLORA_ERR_INVALID_ARG;
   if (!aligned16(W) || !aligned16(codes) || (reinterpret_cast<uintptr_t>(absmax_scale) & 3u))
     return QLORA_ERR_ALIGNMENT;
   if (numel > (int64_t(1) << 46)) return QLORA_ERR_UNSUPPORTED;
   ProfScope p(static_cast<cudaStream_t>(stream), "quantize_nf4", 1);
-  const cudaError_t e = launch_quantize_nf4(W, numel, codes, absmax_q, absmax_scale, nf4_params(),
+  const cudaError_t e = launch_quantize_nf4(W, numel, codes, absmax_q, absmax_scale, *P,
                                             static_cast<cudaStream_t>(stream));
+  p.done();
+  return e == cudaSuccess ? QLORA_OK : cuda_fail(e);
+}
+
+qlora_status qlora_quantize_nf4(const uint16_t* W, int64_t numel, uint8_t* codes, uint8_t* absmax_q,
+                                float* absmax_scale, void* stream) {
+  return qlora_quantize_4bit(W, numel, QLORA_CODE_NF4, codes, absmax_q, absmax_scale, stream);
+}
+
+qlora_status qlora_dequantize_4bit(const uint8_t* codes, const uint8_t* absmax_q, const float* absmax_scale,
+                                   int64_t numel, int32_t code, uint16_t* W_out, void* stream) {
+  if (!codes || !absmax_q || !absmax_scale || !W_out || numel <= 0) return QLORA_ERR_INVALID_ARG;
+  const Nf4Params* P = code_params_or_null(code);
+  if (!P) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(codes) || !aligned16(W_out) || (reinterpret_cast<uintptr_t>(absmax_scale) & 3u))
+    return QLORA_ERR_ALIGNMENT;
+  if (numel > (int64_t(1) << 46)) return QLORA_ERR_UNSUPPORTED;
+  ProfScope p(static_cast<cudaStream_t>(stream), "dequantize_nf4", 1);
+  const cudaError_t e = launch_dequantize_nf4(codes, absmax_q, absmax_scale, numel, W_out, *P,
+                                              static_cast<cudaStream_t>(stream));
   p.done();
   return e == cudaSuccess ? QLORA_OK : cuda_fail(e);
 }
 
 qlora_status qlora_dequantize_nf4(const uint8_t* codes, const uint8_t* absmax_q, const float* absmax_scale,
                                   int64_t numel, uint16_t* W_out, void* stream) {
-  if (!codes || !absmax_q || !absmax_scale || !W_out || numel <= 0) return QLORA_ERR_INVALID_ARG;
-  if (!aligned16(codes) || !aligned16(W_out) || (reinterpret_cast<uintptr_t>(absmax_scale) & 3u))
-    return QLORA_ERR_ALIGNMENT;
-  if (numel > (int64_t(1) << 46)) return QLORA_ERR_UNSUPPORTED;
-  ProfScope p(static_cast<cudaStream_t>(stream), "dequantize_nf4", 1);
-  const cudaError_t e = launch_dequantize_nf4(codes, absmax_q, absmax_scale, numel, W_out, nf4_params(),
-                                              static_cast<cudaStream_t>(stream));
-  p.done();
-  return e == cudaSuccess ? QLORA_OK : cuda_fail(e);
+  return qlora_dequantize_4bit(codes, absmax_q, absmax_scale, numel, QLORA_CODE_NF4, W_out, stream);
 }
 
 size_t qlora_workspace_bytes(int64_t M, int64_t K, int64_t N, int32_t r) {
@@ -176,11 +190,13 @@ size_t qlora_workspace_bytes(int64_t M, int64_t K, int64_t N, int32_t r) {
   return ws_layout(M, K, N, r).total;
 }
 
-qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, int64_t K, int64_t N, const uint8_t* codes,
-                              const uint8_t* absmax_q, const float* absmax_scale, const uint16_t* A,
-                              const uint16_t* B, int32_t r, float scale, uint16_t* Y, float* T_save,
-                              void* workspace, size_t ws_bytes, void* stream) {
+qlora_status qlora_linear_fwd_4bit(const uint16_t* X, int64_t M, int64_t K, int64_t N, const uint8_t* codes,
+                                   const uint8_t* absmax_q, const float* absmax_scale, int32_t code,
+                                   const uint16_t* A, const uint16_t* B, int32_t r, float scale, uint16_t* Y,
+                                   float* T_save, void* workspace, size_t ws_bytes, void* stream) {
   if (!X || !codes || !absmax_q || !absmax_scale || !A || !B || !Y || !T_save) return QLORA_ERR_INVALID_ARG;
+  const Nf4Params* Pc = code_params_or_null(code);
+  if (!Pc) return QLORA_ERR_INVALID_ARG;
   if (!std::isfinite(scale)) return QLORA_ERR_INVALID_ARG;
   const qlora_status sh = check_linear_shape(M, K, N, r);
   if (sh != QLORA_OK) return sh;
@@ -193,7 +209,7 @@ qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, int64_t K, int64_t N
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   int* status = reinterpret_cast<int*>(ws);
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const Nf4Params& P = nf4_params();
+  const Nf4Params& P = *Pc;
 
   uint16_t* Tpair = reinterpret_cast<uint16_t*>(ws + wl.t_off);
 
@@ -215,12 +231,23 @@ qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, int64_t K, int64_t N
   return QLORA_OK;
 }
 
-qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float* T_save, int64_t M, int64_t K,
-                              int64_t N, const uint8_t* codes, const uint8_t* absmax_q, const float* absmax_scale,
-                              const uint16_t* A, const uint16_t* B, int32_t r, float scale, uint16_t* dX, float* dA,
-                              float* dB, void* workspace, size_t ws_bytes, void* stream) {
+qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, int64_t K, int64_t N, const uint8_t* codes,
+                              const uint8_t* absmax_q, const float* absmax_scale, const uint16_t* A,
+                              const uint16_t* B, int32_t r, float scale, uint16_t* Y, float* T_save,
+                              void* workspace, size_t ws_bytes, void* stream) {
+  return qlora_linear_fwd_4bit(X, M, K, N, codes, absmax_q, absmax_scale, QLORA_CODE_NF4, A, B, r, scale, Y, T_save,
+                               workspace, ws_bytes, stream);
+}
+
+qlora_status qlora_linear_bwd_4bit(const uint16_t* dY, const uint16_t* X, const float* T_save, int64_t M, int64_t K,
+                                   int64_t N, const uint8_t* codes, const uint8_t* absmax_q,
+                                   const float* absmax_scale, int32_t code, const uint16_t* A, const uint16_t* B,
+                                   int32_t r, float scale, uint16_t* dX, float* dA, float* dB, void* workspace,
+                                   size_t ws_bytes, void* stream) {
   if (!dY || !X || !T_save || !codes || !absmax_q || !absmax_scale || !A || !B || !dX || !dA || !dB)
     return QLORA_ERR_INVALID_ARG;
+  const Nf4Params* Pc = code_params_or_null(code);
+  if (!Pc) return QLORA_ERR_INVALID_ARG;
   if (!std::isfinite(scale)) return QLORA_ERR_INVALID_ARG;
   const qlora_status sh = check_linear_shape(M, K, N, r);
   if (sh != QLORA_OK) return sh;
@@ -236,7 +263,7 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float
   uint16_t* Tpair = reinterpret_cast<uint16_t*>(ws + wl.t_off);
   uint16_t* Upair = reinterpret_cast<uint16_t*>(ws + wl.u_off);
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const Nf4Params& P = nf4_params();
+  const Nf4Params& P = *Pc;
 
   // One launch: U = s dY B^T (and the bf16 pair of T) in the first units,
   // the dX tiles, and dA = X^T U and dB = T^T dY in units that fill the SMs
@@ -247,6 +274,14 @@ qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float
   p2.done();
   if (e != cudaSuccess) return cuda_fail(e);
   return QLORA_OK;
+}
+
+qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float* T_save, int64_t M, int64_t K,
+                              int64_t N, const uint8_t* codes, const uint8_t* absmax_q, const float* absmax_scale,
+                              const uint16_t* A, const uint16_t* B, int32_t r, float scale, uint16_t* dX, float* dA,
+                              float* dB, void* workspace, size_t ws_bytes, void* stream) {
+  return qlora_linear_bwd_4bit(dY, X, T_save, M, K, N, codes, absmax_q, absmax_scale, QLORA_CODE_NF4, A, B, r, scale,
+                               dX, dA, dB, workspace, ws_bytes, stream);
 }
 
 qlora_status qlora_silu_gate_fwd(const uint16_t* G, const uint16_t* U, uint16_t* H, int64_t n, void* stream) {
@@ -311,6 +346,13 @@ void qlora_nf4_codebook(float out[16]) {
   if (!out) return;
   const Nf4Params& P = nf4_params();
   std::memcpy(out, P.q, sizeof(P.q));
+}
+
+qlora_status qlora_codebook(int32_t code, float out[16]) {
+  const Nf4Params* P = code_params_or_null(code);
+  if (!P || !out) return QLORA_ERR_INVALID_ARG;
+  std::memcpy(out, P->q, sizeof(P->q));
+  return QLORA_OK;
 }
 
 const char* qlora_status_string(qlora_status s) {

@@ -24,9 +24,10 @@ double normal_quantile_upper(double p) {
   return x;
 }
 
-Nf4Params build() {
+// Levels plus the encoder's boundaries for a sorted table of 16 levels.
+Nf4Params with_boundaries(const float q[16]) {
   Nf4Params P{};
-  nf4_levels(P.q);
+  for (int i = 0; i < 16; ++i) P.q[i] = q[i];
   for (int j = 0; j < 15; ++j) {
     const double mid = 0.5 * (static_cast<double>(P.q[j]) + static_cast<double>(P.q[j + 1]));  // exact
     float u = static_cast<float>(mid);
@@ -35,6 +36,35 @@ Nf4Params build() {
     P.bnd[j] = 0.5 * (static_cast<double>(below) + static_cast<double>(u));  // exact (25 bits)
   }
   return P;
+}
+
+Nf4Params build_nf4() {
+  float q[16];
+  nf4_levels(q);
+  return with_boundaries(q);
+}
+
+// FP4: the float with 1 sign, 2 exponent and 1 mantissa bit; its seven
+// non-zero magnitudes 0.5, 1, 1.5, 2, 3, 4, 6 divided by the largest.  Int4:
+// k / 7.  Sorted with the zero at index 7; index 15 repeats +1, so that the
+// nearest-level rule (ties to the lower index) never picks it.
+Nf4Params build_fp4() {
+  const double mags[7] = {0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+  float q[16];
+  for (int i = 0; i < 7; ++i) {
+    q[6 - i] = static_cast<float>(-mags[i] / 6.0);
+    q[8 + i] = static_cast<float>(mags[i] / 6.0);
+  }
+  q[7] = 0.0f;
+  q[15] = q[14];
+  return with_boundaries(q);
+}
+
+Nf4Params build_int4() {
+  float q[16];
+  for (int k = -7; k <= 7; ++k) q[k + 7] = static_cast<float>(k / 7.0);
+  q[15] = q[14];
+  return with_boundaries(q);
 }
 
 }  // namespace
@@ -53,11 +83,19 @@ void nf4_levels(float out[16]) {
   for (int i = 0; i < 16; ++i) out[i] = static_cast<float>(v[i] / top);
 }
 
-const Nf4Params& nf4_params() {
+const Nf4Params& nf4_params() { return code_params(0); }
+
+const Nf4Params* code_params_or_null(int code) {
   static std::once_flag once;
-  static Nf4Params P;
-  std::call_once(once, [] { P = build(); });
-  return P;
+  static Nf4Params P[3];
+  std::call_once(once, [] {
+    P[0] = build_nf4();
+    P[1] = build_fp4();
+    P[2] = build_int4();
+  });
+  return (code >= 0 && code < 3) ? &P[code] : nullptr;
 }
+
+const Nf4Params& code_params(int code) { return *code_params_or_null(code >= 0 && code < 3 ? code : 0); }
 
 }  // namespace qlora

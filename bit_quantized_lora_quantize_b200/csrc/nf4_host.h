@@ -19,4 +19,9 @@ void nf4_levels(float out[16]);
 // j and j + 1.  Computed once per process; thread-safe.
 const Nf4Params& nf4_params();
 
+// The same for each 4-bit code of include/qlora.h (0 NF4, 1 FP4, 2 Int4):
+// null for an unknown code; code_params falls back to NF4.
+const Nf4Params* code_params_or_null(int code);
+const Nf4Params& code_params(int code);
+
 }  // namespace qlora

@@ -18,6 +18,8 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libqlora.so")
 
 QLORA_OK = 0
+# 4-bit codes of the packed format (qlora_code in include/qlora.h).
+CODES = {"nf4": 0, "fp4": 1, "int4": 2}
 STATUS_NAMES = {0: "QLORA_OK", 1: "QLORA_ERR_INVALID_ARG", 2: "QLORA_ERR_ALIGNMENT", 3: "QLORA_ERR_UNSUPPORTED",
                 4: "QLORA_ERR_WORKSPACE", 5: "QLORA_ERR_CUDA", 6: "QLORA_ERR_TIMEOUT"}
 
@@ -27,6 +29,14 @@ _I64 = ctypes.c_int64
 _SIGS = {
     "qlora_quantize_nf4": (ctypes.c_int, [_P, _I64, _P, _P, _P, _P]),
     "qlora_dequantize_nf4": (ctypes.c_int, [_P, _P, _P, _I64, _P, _P]),
+    "qlora_quantize_4bit": (ctypes.c_int, [_P, _I64, ctypes.c_int32, _P, _P, _P, _P]),
+    "qlora_dequantize_4bit": (ctypes.c_int, [_P, _P, _P, _I64, ctypes.c_int32, _P, _P]),
+    "qlora_linear_fwd_4bit": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, ctypes.c_int32, _P, _P,
+                                             ctypes.c_int32, ctypes.c_float, _P, _P, _P, ctypes.c_size_t, _P]),
+    "qlora_linear_bwd_4bit": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _I64, _P, _P, _P, ctypes.c_int32, _P, _P,
+                                             ctypes.c_int32, ctypes.c_float, _P, _P, _P, _P, ctypes.c_size_t,
+                                             _P]),
+    "qlora_codebook": (ctypes.c_int, [ctypes.c_int32, ctypes.POINTER(ctypes.c_float)]),
     "qlora_linear_fwd": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, ctypes.c_int32, ctypes.c_float,
                                         _P, _P, _P, ctypes.c_size_t, _P]),
     "qlora_linear_bwd": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P, _P, ctypes.c_int32,
@@ -35,6 +45,12 @@ _SIGS = {
                                                 ctypes.c_float, _P, _P, _P]),
     "qlora_silu_gate_fwd": (ctypes.c_int, [_P, _P, _P, _I64, _P]),
     "qlora_silu_gate_bwd": (ctypes.c_int, [_P, _P, _P, _P, _P, _I64, _P]),
+    "qlora_paged_malloc": (ctypes.c_void_p, [ctypes.c_size_t, ctypes.c_int, _P]),
+    "qlora_paged_free": (None, [_P, ctypes.c_size_t, ctypes.c_int, _P]),
+    "qlora_paged_prefetch": (ctypes.c_int, [_P, ctypes.c_size_t, ctypes.c_int32, _P]),
+    "qlora_paged_location": (ctypes.c_int, [_P, ctypes.c_size_t, ctypes.POINTER(ctypes.c_int32)]),
+    "qlora_adamw_step": (ctypes.c_int, [_P, _P, _P, _P, _P, _I64, ctypes.c_int32, ctypes.c_float, ctypes.c_float,
+                                        ctypes.c_float, ctypes.c_float, ctypes.c_float, _P]),
     "qlora_workspace_bytes": (ctypes.c_size_t, [_I64, _I64, _I64, ctypes.c_int32]),
     "qlora_check_status": (ctypes.c_int, [_P, _P]),
     "qlora_set_wait_timeout": (ctypes.c_int, [ctypes.c_uint64]),
@@ -101,12 +117,14 @@ def _stream() -> int:
 # ---------------------------------------------------------------- packed weight
 @dataclass
 class PackedNF4:
-    """A frozen weight [N, K] in the packed NF4 format of include/qlora.h."""
+    """A frozen weight [N, K] in the packed format of include/qlora.h, with
+    the NF4 levels (or the FP4 / Int4 ones, ``code``)."""
 
     codes: torch.Tensor         # uint8 [ceil(N*K/2)]
     absmax_q: torch.Tensor      # uint8 [NB]
     absmax_scale: torch.Tensor  # float32 [NB2]
     shape: tuple
+    code: str = "nf4"
 
     @property
     def numel(self) -> int:
@@ -127,10 +145,16 @@ def qlora_nf4_codebook() -> list:
     return list(buf)
 
 
-def qlora_quantize_nf4(W: torch.Tensor, out: PackedNF4 = None) -> PackedNF4:
-    """Quantize a bf16 CUDA tensor (any shape, flattened row-major).  `out`,
-    if given, is a PackedNF4 of the same element count whose buffers are
-    overwritten."""
+def qlora_codebook(code: str = "nf4") -> list:
+    buf = (ctypes.c_float * 16)()
+    _check("qlora_codebook", lib().qlora_codebook(CODES[code], buf))
+    return list(buf)
+
+
+def qlora_quantize_nf4(W: torch.Tensor, out: PackedNF4 = None, code: str = "nf4") -> PackedNF4:
+    """Quantize a bf16 CUDA tensor (any shape, flattened row-major) with the
+    NF4 levels (or ``code`` = "fp4" / "int4").  `out`, if given, is a
+    PackedNF4 of the same element count whose buffers are overwritten."""
     _require_cuda(W)
     if W.dtype != torch.bfloat16:
         raise ValueError("W must be bfloat16")
@@ -146,8 +170,13 @@ def qlora_quantize_nf4(W: torch.Tensor, out: PackedNF4 = None) -> PackedNF4:
         if (codes.numel(), aq.numel(), sc.numel()) != (nc, nb, nb2):
             raise ValueError("out does not hold a weight of this size")
         _require_cuda(codes, aq, sc)
-    _check("qlora_quantize_nf4", lib().qlora_quantize_nf4(_ptr(W), n, _ptr(codes), _ptr(aq), _ptr(sc), _stream()))
-    return PackedNF4(codes, aq, sc, tuple(W.shape))
+    if code == "nf4":
+        _check("qlora_quantize_nf4", lib().qlora_quantize_nf4(_ptr(W), n, _ptr(codes), _ptr(aq), _ptr(sc),
+                                                              _stream()))
+    else:
+        _check("qlora_quantize_4bit", lib().qlora_quantize_4bit(_ptr(W), n, CODES[code], _ptr(codes), _ptr(aq),
+                                                                _ptr(sc), _stream()))
+    return PackedNF4(codes, aq, sc, tuple(W.shape), code)
 
 
 def qlora_dequantize_nf4(p: PackedNF4, out: torch.Tensor = None) -> torch.Tensor:
@@ -156,8 +185,13 @@ def qlora_dequantize_nf4(p: PackedNF4, out: torch.Tensor = None) -> torch.Tensor
         out = torch.empty(p.shape, dtype=torch.bfloat16, device=p.codes.device)
     elif out.dtype != torch.bfloat16 or out.numel() != p.numel or not out.is_contiguous():
         raise ValueError("out must be a contiguous bf16 tensor of the weight's size")
-    _check("qlora_dequantize_nf4", lib().qlora_dequantize_nf4(_ptr(p.codes), _ptr(p.absmax_q), _ptr(p.absmax_scale),
-                                                              p.numel, _ptr(out), _stream()))
+    if p.code == "nf4":
+        _check("qlora_dequantize_nf4", lib().qlora_dequantize_nf4(_ptr(p.codes), _ptr(p.absmax_q),
+                                                                  _ptr(p.absmax_scale), p.numel, _ptr(out), _stream()))
+    else:
+        _check("qlora_dequantize_4bit", lib().qlora_dequantize_4bit(_ptr(p.codes), _ptr(p.absmax_q),
+                                                                    _ptr(p.absmax_scale), p.numel, CODES[p.code],
+                                                                    _ptr(out), _stream()))
     return out
 
 
@@ -187,9 +221,14 @@ def qlora_linear_fwd(X: torch.Tensor, W: PackedNF4, A: torch.Tensor, B: torch.Te
         Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
     if T_save is None:
         T_save = torch.empty(M, r, dtype=torch.float32, device=dev)
-    _check("qlora_linear_fwd", lib().qlora_linear_fwd(
-        _ptr(X), M, K, N, _ptr(W.codes), _ptr(W.absmax_q), _ptr(W.absmax_scale), _ptr(A), _ptr(B), r,
-        float(scale), _ptr(Y), _ptr(T_save), _ptr(workspace), workspace.numel(), _stream()))
+    if W.code == "nf4":
+        _check("qlora_linear_fwd", lib().qlora_linear_fwd(
+            _ptr(X), M, K, N, _ptr(W.codes), _ptr(W.absmax_q), _ptr(W.absmax_scale), _ptr(A), _ptr(B), r,
+            float(scale), _ptr(Y), _ptr(T_save), _ptr(workspace), workspace.numel(), _stream()))
+    else:
+        _check("qlora_linear_fwd_4bit", lib().qlora_linear_fwd_4bit(
+            _ptr(X), M, K, N, _ptr(W.codes), _ptr(W.absmax_q), _ptr(W.absmax_scale), CODES[W.code], _ptr(A),
+            _ptr(B), r, float(scale), _ptr(Y), _ptr(T_save), _ptr(workspace), workspace.numel(), _stream()))
     return Y, T_save
 
 
@@ -197,6 +236,8 @@ def qlora_linear_fwd_noalloc(X: torch.Tensor, W: PackedNF4, A: torch.Tensor, B: 
                              Y: torch.Tensor, T_save: torch.Tensor):
     """Forward into caller-provided Y and T_save with no workspace: the
     library takes its scratch from a fixed device array (see include/qlora.h)."""
+    if W.code != "nf4":
+        raise ValueError("the allocation-free forward takes NF4 weights only")
     M, K = X.shape
     N = W.shape[0]
     r = A.shape[1]
@@ -224,9 +265,16 @@ def qlora_linear_bwd(dY: torch.Tensor, X: torch.Tensor, T_save: torch.Tensor, W:
         dA = torch.empty(K, r, dtype=torch.float32, device=dev)
     if dB is None:
         dB = torch.empty(r, N, dtype=torch.float32, device=dev)
-    _check("qlora_linear_bwd", lib().qlora_linear_bwd(
-        _ptr(dY), _ptr(X), _ptr(T_save), M, K, N, _ptr(W.codes), _ptr(W.absmax_q), _ptr(W.absmax_scale), _ptr(A),
-        _ptr(B), r, float(scale), _ptr(dX), _ptr(dA), _ptr(dB), _ptr(workspace), workspace.numel(), _stream()))
+    if W.code == "nf4":
+        _check("qlora_linear_bwd", lib().qlora_linear_bwd(
+            _ptr(dY), _ptr(X), _ptr(T_save), M, K, N, _ptr(W.codes), _ptr(W.absmax_q), _ptr(W.absmax_scale),
+            _ptr(A), _ptr(B), r, float(scale), _ptr(dX), _ptr(dA), _ptr(dB), _ptr(workspace), workspace.numel(),
+            _stream()))
+    else:
+        _check("qlora_linear_bwd_4bit", lib().qlora_linear_bwd_4bit(
+            _ptr(dY), _ptr(X), _ptr(T_save), M, K, N, _ptr(W.codes), _ptr(W.absmax_q), _ptr(W.absmax_scale),
+            CODES[W.code], _ptr(A), _ptr(B), r, float(scale), _ptr(dX), _ptr(dA), _ptr(dB), _ptr(workspace),
+            workspace.numel(), _stream()))
     return dX, dA, dB
 
 
@@ -291,7 +339,7 @@ def qlora_profile_stop(max_entries: int = 32) -> dict:
     return out
 
 
-__all__ = ["qlora_profile_start", "qlora_profile_stop", "LIB_PATH", "lib", "QloraError", "PackedNF4", "packed_sizes", "qlora_nf4_codebook", "qlora_quantize_nf4",
+__all__ = ["CODES", "qlora_codebook", "qlora_profile_start", "qlora_profile_stop", "LIB_PATH", "lib", "QloraError", "PackedNF4", "packed_sizes", "qlora_nf4_codebook", "qlora_quantize_nf4",
            "qlora_dequantize_nf4", "qlora_workspace_bytes", "new_workspace", "qlora_linear_fwd", "qlora_linear_bwd",
            "qlora_linear_fwd_noalloc",
            "qlora_check_status", "qlora_set_wait_timeout", "qlora_get_wait_timeout", "qlora_silu_gate_fwd",

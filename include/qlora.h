@@ -72,6 +72,22 @@ typedef enum {
 } qlora_status;
 
 /*
+ * 4-bit codes of the packed format.  NF4 is the method's type; FP4 and Int4
+ * are the two 4-bit types the pages compare it with ("1. 4-bit NormalFloat
+ * (NF4)": Integer 4-bit and Float 4-bit, with NF4 the lower-error one;
+ * "Performance and Evaluation", "NF4 efficiency").  The pages define neither;
+ * this library reads them as
+ *   QLORA_CODE_FP4   the float with 1 sign, 2 exponent and 1 mantissa bit
+ *                    (magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6) divided by 6,
+ *   QLORA_CODE_INT4  the symmetric integer code k / 7, k = -7..7.
+ * Both keep everything else of the packed format (blocks of 64, double
+ * quantization, nibble order, zero level at index 7).  Their 15 distinct
+ * levels fill indices 0..14 in ascending order and index 15 repeats +1; the
+ * nearest-level rule (ties to the lower index) never produces code 15.
+ */
+typedef enum { QLORA_CODE_NF4 = 0, QLORA_CODE_FP4 = 1, QLORA_CODE_INT4 = 2 } qlora_code;
+
+/*
  * Blockwise NF4 quantization with double-quantized constants.
  * "AI Glossary: QLoRA", second paragraph; "1. 4-bit NormalFloat (NF4)" and
  * "2. Double Quantization" in "QLoRA: Fine-Tuning 65-Billion Parameter
@@ -88,6 +104,12 @@ typedef enum {
 QLORA_API qlora_status qlora_quantize_nf4(const uint16_t* W, int64_t numel, uint8_t* codes, uint8_t* absmax_q,
                                 float* absmax_scale, void* stream);
 
+/* The same quantization with the levels of `code` (a qlora_code; any other
+ * value returns QLORA_ERR_INVALID_ARG).  qlora_quantize_nf4 is this call
+ * with QLORA_CODE_NF4. */
+QLORA_API qlora_status qlora_quantize_4bit(const uint16_t* W, int64_t numel, int32_t code, uint8_t* codes,
+                                           uint8_t* absmax_q, float* absmax_scale, void* stream);
+
 /*
  * Dequantization to bf16 (the weight the linear calls multiply by).
  * "AI Glossary: QLoRA", second paragraph (4-bit weights turned back into
@@ -97,6 +119,11 @@ QLORA_API qlora_status qlora_quantize_nf4(const uint16_t* W, int64_t numel, uint
  */
 QLORA_API qlora_status qlora_dequantize_nf4(const uint8_t* codes, const uint8_t* absmax_q, const float* absmax_scale,
                                   int64_t numel, uint16_t* W_out, void* stream);
+
+/* Dequantization of a weight packed with the levels of `code`. */
+QLORA_API qlora_status qlora_dequantize_4bit(const uint8_t* codes, const uint8_t* absmax_q,
+                                             const float* absmax_scale, int64_t numel, int32_t code,
+                                             uint16_t* W_out, void* stream);
 
 /*
  * Forward of the frozen-NF4 linear layer with a LoRA adapter.
@@ -136,6 +163,13 @@ QLORA_API qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, int64_t K,
                               const uint16_t* B, int32_t r, float scale, uint16_t* Y, float* T_save,
                               void* workspace, size_t ws_bytes, void* stream);
 
+/* qlora_linear_fwd for a weight packed with the levels of `code`. */
+QLORA_API qlora_status qlora_linear_fwd_4bit(const uint16_t* X, int64_t M, int64_t K, int64_t N,
+                                             const uint8_t* codes, const uint8_t* absmax_q,
+                                             const float* absmax_scale, int32_t code, const uint16_t* A,
+                                             const uint16_t* B, int32_t r, float scale, uint16_t* Y, float* T_save,
+                                             void* workspace, size_t ws_bytes, void* stream);
+
 /*
  * Backward of the same layer for an upstream gradient dY.  Gradients are
  * produced only for the adapter; the frozen base weight gets none
@@ -158,6 +192,13 @@ QLORA_API qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, c
                               int64_t N, const uint8_t* codes, const uint8_t* absmax_q, const float* absmax_scale,
                               const uint16_t* A, const uint16_t* B, int32_t r, float scale, uint16_t* dX, float* dA,
                               float* dB, void* workspace, size_t ws_bytes, void* stream);
+
+/* qlora_linear_bwd for a weight packed with the levels of `code`. */
+QLORA_API qlora_status qlora_linear_bwd_4bit(const uint16_t* dY, const uint16_t* X, const float* T_save, int64_t M,
+                                             int64_t K, int64_t N, const uint8_t* codes, const uint8_t* absmax_q,
+                                             const float* absmax_scale, int32_t code, const uint16_t* A,
+                                             const uint16_t* B, int32_t r, float scale, uint16_t* dX, float* dA,
+                                             float* dB, void* workspace, size_t ws_bytes, void* stream);
 
 /*
  * qlora_linear_fwd without a workspace argument, for callers that cannot
@@ -211,6 +252,42 @@ QLORA_API qlora_status qlora_silu_gate_fwd(const uint16_t* G, const uint16_t* U,
 QLORA_API qlora_status qlora_silu_gate_bwd(const uint16_t* G, const uint16_t* U, const uint16_t* dH, uint16_t* dG,
                                            uint16_t* dU, int64_t n, void* stream);
 
+/*
+ * Paged optimizer for the LoRA parameters.  "3. Paged Optimizers" and "AI
+ * Glossary: QLoRA", second paragraph: only the LoRA matrices are trained,
+ * and their optimizer states live in NVIDIA unified memory so that they can
+ * move between GPU and CPU memory during memory spikes.
+ *
+ * qlora_paged_malloc / qlora_paged_free: unified (managed) memory for the
+ * optimizer states, with the allocate/free signatures of PyTorch's pluggable
+ * allocator (size, device, stream) / (ptr, size, device, stream).  These are
+ * the only calls of this library that allocate; the memory belongs to the
+ * caller.  malloc returns NULL on failure (qlora_last_cuda_error says why).
+ * free synchronises `stream` (if any) before releasing the memory.
+ *
+ * qlora_paged_prefetch: asynchronously moves [ptr, ptr + bytes) to the
+ * current device (to_device != 0) or to host memory (to_device == 0) on
+ * `stream`.  Kernels may touch the memory wherever it is: pages that are on
+ * the host migrate on demand.  qlora_paged_location reports where the range
+ * was last prefetched (a device index, or -1 for the host).
+ *
+ * qlora_adamw_step: one AdamW step over n float32 parameters, in place:
+ *   m = b1 m + (1 - b1) g;  v = b2 v + (1 - b2) g^2
+ *   p = p - lr (m / (1 - b1^step) / (sqrt(v / (1 - b2^step)) + eps) + wd p)
+ * step >= 1 counts the steps taken so far including this one; m and v start
+ * at zero.  param_bf16 (may be NULL) receives bf16_rne(p), the adapter the
+ * linear calls read.  param, grad, m, v: float[n], 4-byte aligned (16-byte
+ * alignment takes the vector path); param_bf16 2-byte aligned.  The step is
+ * the textbook AdamW; the pages name no optimizer formula.
+ */
+QLORA_API void* qlora_paged_malloc(size_t size, int device, void* stream);
+QLORA_API void qlora_paged_free(void* ptr, size_t size, int device, void* stream);
+QLORA_API qlora_status qlora_paged_prefetch(const void* ptr, size_t bytes, int32_t to_device, void* stream);
+QLORA_API qlora_status qlora_paged_location(const void* ptr, size_t bytes, int32_t* location);
+QLORA_API qlora_status qlora_adamw_step(float* param, uint16_t* param_bf16, const float* grad, float* m, float* v,
+                                        int64_t n, int32_t step, float lr, float beta1, float beta2, float eps,
+                                        float weight_decay, void* stream);
+
 /* Workspace bytes needed by qlora_linear_fwd / qlora_linear_bwd for these sizes
  * (0 for an unsupported shape). */
 QLORA_API size_t qlora_workspace_bytes(int64_t M, int64_t K, int64_t N, int32_t r);
@@ -236,6 +313,9 @@ QLORA_API uint64_t qlora_get_wait_timeout(void);
 
 /* The 16 NF4 levels (float32, ascending) this library encodes against. */
 QLORA_API void qlora_nf4_codebook(float out[16]);
+
+/* The 16 levels of `code` (float32, ascending; see qlora_code). */
+QLORA_API qlora_status qlora_codebook(int32_t code, float out[16]);
 
 /* Static description of a status code. */
 QLORA_API const char* qlora_status_string(qlora_status s);

@@ -45,6 +45,35 @@ def test_codebook_matches_oracle_in_float32(L):
     np.testing.assert_array_equal(np.array(q.qlora_nf4_codebook(), dtype=np.float32), nf4_codebook())
 
 
+@pytest.mark.parametrize("code", ["nf4", "fp4", "int4"])
+def test_every_codebook_matches_oracle_in_float32(L, code):
+    from oracle import codebook
+    np.testing.assert_array_equal(np.array(q.qlora_codebook(code), dtype=np.float32), codebook(code))
+
+
+def test_unknown_code_is_rejected(L):
+    buf = (ctypes.c_float * 16)()
+    assert L.qlora_codebook(3, buf) == 1
+    assert L.qlora_quantize_4bit(FAKE, 64, 7, FAKE, FAKE, FAKE, None) == 1
+    assert L.qlora_dequantize_4bit(FAKE, FAKE, FAKE, 64, -1, FAKE, None) == 1
+
+
+def test_adamw_validation(L):
+    P = FAKE
+    args = dict(n=10, step=1, lr=1e-3, b1=0.9, b2=0.999, eps=1e-8, wd=0.0)
+
+    def call(p=P, **kw):
+        a = dict(args, **kw)
+        return L.qlora_adamw_step(p, None, P, P, P, a["n"], a["step"], a["lr"], a["b1"], a["b2"], a["eps"], a["wd"],
+                                  None)
+    assert call(step=0) == 1            # steps count from 1
+    assert call(n=0) == 1
+    assert call(b1=1.0) == 1 and call(b2=-0.1) == 1
+    assert call(lr=float("inf")) == 1
+    assert call(p=P + 2) == 2           # float buffers must be 4-byte aligned
+    assert L.qlora_paged_prefetch(None, 16, 1, None) == 1
+
+
 def test_status_strings(L):
     for s in range(7):
         assert L.qlora_status_string(s)
