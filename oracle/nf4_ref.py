@@ -45,6 +45,20 @@ What the pages fix, and the readings taken where they are silent:
   indices 0..14 with the zero at index 7, and index 15 repeats the top level
   +1.  Ties go to the lower index, so code 15 is never produced and every
   code's value is the index's level, as for NF4.
+* "2. Double Quantization" says only that the constants are quantized.  A
+  second reading (``dq="centred_fp8"``; the original QLoRA paper's variant,
+  not printed on the pages) codes them with an 8-bit float after removing
+  their mean, since the constants are all positive:
+    mu  = fp32(exact mean of all block absmaxes c_b of the tensor)
+    d_b = fp32(c_b - mu)
+    s_g = fp32(max |d_b| over the 256-group / 448)       (448: E4M3's largest)
+    k_b = the E4M3 code (1 sign, 4 exponent bits with bias 7, 3 mantissa
+          bits; no infinities) nearest to fp32(d_b / s_g), ties to the even
+          code, saturating at +-448; a negative value that rounds to zero
+          gives -0 (code 0x80); k_b = 0 when s_g = 0
+    a'  = fp32(fp32(E4M3(k_b) * s_g) + mu)
+  Stored: k_b in absmax_q, s_g per group in absmax_scale, then mu as one
+  extra float at the end (NB2 + 1 floats).  Level 1 still uses the true c_b.
 """
 
 from __future__ import annotations
@@ -139,9 +153,65 @@ def _level2_table() -> np.ndarray:
     return (np.arange(256, dtype=np.float64) / 255.0).astype(np.float32)
 
 
-def quantize_nf4(w: np.ndarray, block: int = BLOCK, group: int = GROUP, code: str = "nf4"):
+def e4m3_value(code: int) -> float:
+    """Value of an 8-bit E4M3 code (NaN for the two NaN codes)."""
+    sign = -1.0 if code & 0x80 else 1.0
+    e, m = (code >> 3) & 0xF, code & 0x7
+    if e == 0xF and m == 0x7:
+        return float("nan")
+    if e == 0:
+        return sign * m * 2.0 ** -9
+    return sign * (1.0 + m / 8.0) * 2.0 ** (e - 7)
+
+
+def e4m3_encode(x: np.ndarray) -> np.ndarray:
+    """Nearest E4M3 code of each float32 value, ties to the even code,
+    saturating at +-448; the sign of a negative value is kept (-0 = 0x80)."""
+    mags = np.array([e4m3_value(k) for k in range(0x7F)], dtype=np.float64)  # codes 0..126, ascending
+    x = np.asarray(x, dtype=np.float64).reshape(-1)
+    a = np.minimum(np.abs(x), 448.0)
+    hi = np.searchsorted(mags, a, side="left")          # first level >= a
+    hi = np.minimum(hi, len(mags) - 1)
+    lo = np.maximum(hi - 1, 0)
+    dlo, dhi = a - mags[lo], mags[hi] - a
+    code = np.where(dhi < dlo, hi, lo)
+    tie = (dhi == dlo) & (hi != lo)
+    code = np.where(tie, np.where(lo % 2 == 0, lo, hi), code)
+    code = np.where(a == mags[hi], hi, code)
+    return (code | np.where(np.signbit(x), 0x80, 0)).astype(np.uint8)
+
+
+def _rn_f32_ratio(num: int, den: int) -> np.float32:
+    """float32 nearest (ties to even) to the non-negative rational num/den."""
+    if num == 0:
+        return np.float32(0.0)
+    # exponent e with 2^e <= num/den < 2^(e+1)
+    e = num.bit_length() - den.bit_length()
+    if (num << max(0, -e)) < (den << max(0, e)):
+        e -= 1
+    q = max(e, -126) - 23  # quantum of the result's binade (subnormals at 2^-149)
+    if q >= 0:
+        n, d = num, den << q
+    else:
+        n, d = num << -q, den
+    m, r = divmod(n, d)
+    if 2 * r > d or (2 * r == d and m % 2 == 1):
+        m += 1
+    return np.float32(m * 2.0 ** q)
+
+
+def centred_mean(c: np.ndarray) -> np.float32:
+    """fp32 of the exact mean of the block absmaxes (each a bf16 value)."""
+    ints = (np.asarray(c, dtype=np.float64) * 2.0 ** 133)  # exact integers: bf16 values are multiples of 2^-133
+    total = sum(int(v) for v in ints.tolist())
+    return _rn_f32_ratio(total, len(ints) << 133)
+
+
+def quantize_nf4(w: np.ndarray, block: int = BLOCK, group: int = GROUP, code: str = "nf4", dq: str = "linear8"):
     """Blockwise NF4 quantization with double-quantized constants (or the
-    same scheme with the FP4 or Int4 levels, ``code`` = "fp4" / "int4").
+    same scheme with the FP4 or Int4 levels, ``code`` = "fp4" / "int4"; the
+    constants coded as in the module header, ``dq`` = "linear8" or
+    "centred_fp8").
 
     ``w``: any-shape array of bfloat16 values (given as float32/float64 that
     lie on the bf16 grid), flattened row-major.
@@ -186,9 +256,24 @@ def quantize_nf4(w: np.ndarray, block: int = BLOCK, group: int = GROUP, code: st
     packed = ((pairs[:, 0] << 4) | pairs[:, 1]).astype(np.uint8)
     packed = packed[: (n + 1) // 2]
 
+    nb2 = -(-nb // group)
+    if dq == "centred_fp8":
+        mu = centred_mean(c)
+        d = (c.astype(np.float64) - np.float64(mu)).astype(np.float32)
+        dpad = np.zeros(nb2 * group, dtype=np.float32)
+        dpad[:nb] = np.abs(d)
+        c1 = dpad.reshape(nb2, group).max(axis=1).astype(np.float32)
+        sg = (c1.astype(np.float64) / 448.0).astype(np.float32)
+        sb = np.repeat(sg, group)[:nb]
+        with np.errstate(invalid="ignore", divide="ignore"):
+            n2 = (d.astype(np.float64) / sb.astype(np.float64)).astype(np.float32)
+        code2 = np.where(sb == 0, np.uint8(0), e4m3_encode(np.where(sb == 0, 0.0, n2))).astype(np.uint8)
+        return packed, code2, np.concatenate([sg, [mu]]).astype(np.float32)
+    if dq != "linear8":
+        raise ValueError(dq)
+
     # Level 2: groups of 256 constants; c1 = max; code2 = nearest k/255 to
     # fp32(c_b / c1); code 0 when c1 == 0.
-    nb2 = -(-nb // group)
     cpad = np.zeros(nb2 * group, dtype=np.float32)
     cpad[:nb] = c
     c1 = cpad.reshape(nb2, group).max(axis=1).astype(np.float32)
@@ -200,16 +285,26 @@ def quantize_nf4(w: np.ndarray, block: int = BLOCK, group: int = GROUP, code: st
     return packed, code2, c1
 
 
-def dequantize_scales(absmax_q: np.ndarray, absmax_scale: np.ndarray, group: int = GROUP) -> np.ndarray:
-    """Per-block dequantized constant a' = fp32(fp32(k/255) * c1), float32[NB]."""
+def dequantize_scales(absmax_q: np.ndarray, absmax_scale: np.ndarray, group: int = GROUP,
+                      dq: str = "linear8") -> np.ndarray:
+    """Per-block dequantized constant a' = fp32(fp32(k/255) * c1), float32[NB]
+    (``dq`` = "centred_fp8": a' = fp32(fp32(E4M3(k) * s_g) + mu))."""
     k = np.asarray(absmax_q, dtype=np.uint8)
+    if dq == "centred_fp8":
+        sc = np.asarray(absmax_scale, dtype=np.float32)
+        mu = np.float64(sc[-1])
+        v = np.array([e4m3_value(int(x)) for x in range(256)], dtype=np.float64)[k]
+        sg = np.repeat(sc[:-1], group)[: k.size].astype(np.float64)
+        p1 = (v * sg).astype(np.float32).astype(np.float64)  # exact product, one rounding
+        return (p1 + mu).astype(np.float32)                   # exact sum, one rounding
     lvl = _level2_table()[k].astype(np.float64)
     c1 = np.repeat(np.asarray(absmax_scale, dtype=np.float32), group)[: k.size].astype(np.float64)
     return (lvl * c1).astype(np.float32)  # exact float64 product, one rounding
 
 
 def dequantize_nf4(codes: np.ndarray, absmax_q: np.ndarray, absmax_scale: np.ndarray,
-                   numel: int, block: int = BLOCK, group: int = GROUP, code: str = "nf4") -> np.ndarray:
+                   numel: int, block: int = BLOCK, group: int = GROUP, code: str = "nf4",
+                   dq: str = "linear8") -> np.ndarray:
     """Dequantize to bfloat16 values (returned as float32 on the bf16 grid).
 
     w' = bf16(fp32(q_code * a')), a' from :func:`dequantize_scales`.
@@ -220,7 +315,7 @@ def dequantize_nf4(codes: np.ndarray, absmax_q: np.ndarray, absmax_scale: np.nda
     nib[1::2] = packed & 0xF
     nib = nib[:numel]
     q = codebook(code).astype(np.float64)
-    a = dequantize_scales(absmax_q, absmax_scale, group)
+    a = dequantize_scales(absmax_q, absmax_scale, group, dq)
     ab = np.repeat(a, block)[:numel].astype(np.float64)
     w32 = (q[nib] * ab).astype(np.float32)  # exact float64 product, one rounding
     return bf16_round(w32)
@@ -280,7 +375,7 @@ def max_half_gap(code: str = "nf4") -> float:
 
 __all__ = [
     "BLOCK", "GROUP", "ZERO_CODE", "nf4_codebook", "fp4_codebook", "int4_codebook", "CODEBOOKS", "codebook",
-    "bf16_round", "bf16_bits",
+    "bf16_round", "bf16_bits", "e4m3_value", "e4m3_encode", "centred_mean",
     "quantize_nf4", "dequantize_scales", "dequantize_nf4", "dequantize_at", "bits_per_parameter",
     "max_half_gap",
 ]
