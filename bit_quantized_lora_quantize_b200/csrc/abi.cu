@@ -95,6 +95,17 @@ cudaEvent_t prof_event() {
 
 }  // namespace
 
+// The levels and constant scheme of a qlora_code value (4-bit code in the
+// low byte, QLORA_DQ_CENTRED_FP8 as a flag); false for an unknown value.
+bool resolve_code(int32_t code, Nf4Params* P) {
+  if (code & ~(0xFF | QLORA_DQ_CENTRED_FP8)) return false;
+  const Nf4Params* base = code_params_or_null(code & 0xFF);
+  if (!base) return false;
+  *P = *base;
+  P->centred = (code & QLORA_DQ_CENTRED_FP8) ? 1 : 0;
+  return true;
+}
+
 qlora_status cuda_fail(cudaError_t e) {
   g_last_cuda_error = cudaGetErrorString(e);
   return QLORA_ERR_CUDA;
@@ -148,12 +159,14 @@ extern "C" {
 qlora_status qlora_quantize_4bit(const uint16_t* W, int64_t numel, int32_t code, uint8_t* codes, uint8_t* absmax_q,
                                  float* absmax_scale, void* stream) {
   if (!W || !codes || !absmax_q || !absmax_scale || numel <= 0) return QLORA_ERR_INVALID_ARG;
-  const Nf4Params* P = code_params_or_null(code);
-  if (!P) return QLORA_ERR_INVALID_ARG;
+  Nf4Params Pv;
+  if (!resolve_code(code, &Pv)) return QLORA_ERR_INVALID_ARG;
+  const Nf4Params* P = &Pv;
   if (!aligned16(W) || !aligned16(codes) || (reinterpret_cast<uintptr_t>(absmax_scale) & 3u))
     return QLORA_ERR_ALIGNMENT;
   if (numel > (int64_t(1) << 46)) return QLORA_ERR_UNSUPPORTED;
-  ProfScope p(static_cast<cudaStream_t>(stream), "quantize_nf4", 1);
+  if (Pv.centred && numel > (int64_t(1) << 38)) return QLORA_ERR_UNSUPPORTED;  // the mean divides by NB < 2^32
+  ProfScope p(static_cast<cudaStream_t>(stream), "quantize_nf4", Pv.centred ? 3 : 1);
   const cudaError_t e = launch_quantize_nf4(W, numel, codes, absmax_q, absmax_scale, *P,
                                             static_cast<cudaStream_t>(stream));
   p.done();
@@ -168,8 +181,9 @@ qlora_status qlora_quantize_nf4(const uint16_t* W, int64_t numel, uint8_t* codes
 qlora_status qlora_dequantize_4bit(const uint8_t* codes, const uint8_t* absmax_q, const float* absmax_scale,
                                    int64_t numel, int32_t code, uint16_t* W_out, void* stream) {
   if (!codes || !absmax_q || !absmax_scale || !W_out || numel <= 0) return QLORA_ERR_INVALID_ARG;
-  const Nf4Params* P = code_params_or_null(code);
-  if (!P) return QLORA_ERR_INVALID_ARG;
+  Nf4Params Pv;
+  if (!resolve_code(code, &Pv)) return QLORA_ERR_INVALID_ARG;
+  const Nf4Params* P = &Pv;
   if (!aligned16(codes) || !aligned16(W_out) || (reinterpret_cast<uintptr_t>(absmax_scale) & 3u))
     return QLORA_ERR_ALIGNMENT;
   if (numel > (int64_t(1) << 46)) return QLORA_ERR_UNSUPPORTED;
@@ -195,8 +209,9 @@ qlora_status qlora_linear_fwd_4bit(const uint16_t* X, int64_t M, int64_t K, int6
                                    const uint16_t* A, const uint16_t* B, int32_t r, float scale, uint16_t* Y,
                                    float* T_save, void* workspace, size_t ws_bytes, void* stream) {
   if (!X || !codes || !absmax_q || !absmax_scale || !A || !B || !Y || !T_save) return QLORA_ERR_INVALID_ARG;
-  const Nf4Params* Pc = code_params_or_null(code);
-  if (!Pc) return QLORA_ERR_INVALID_ARG;
+  Nf4Params Pv;
+  if (!resolve_code(code, &Pv)) return QLORA_ERR_INVALID_ARG;
+  const Nf4Params* Pc = &Pv;
   if (!std::isfinite(scale)) return QLORA_ERR_INVALID_ARG;
   const qlora_status sh = check_linear_shape(M, K, N, r);
   if (sh != QLORA_OK) return sh;
@@ -246,8 +261,9 @@ qlora_status qlora_linear_bwd_4bit(const uint16_t* dY, const uint16_t* X, const 
                                    size_t ws_bytes, void* stream) {
   if (!dY || !X || !T_save || !codes || !absmax_q || !absmax_scale || !A || !B || !dX || !dA || !dB)
     return QLORA_ERR_INVALID_ARG;
-  const Nf4Params* Pc = code_params_or_null(code);
-  if (!Pc) return QLORA_ERR_INVALID_ARG;
+  Nf4Params Pv;
+  if (!resolve_code(code, &Pv)) return QLORA_ERR_INVALID_ARG;
+  const Nf4Params* Pc = &Pv;
   if (!std::isfinite(scale)) return QLORA_ERR_INVALID_ARG;
   const qlora_status sh = check_linear_shape(M, K, N, r);
   if (sh != QLORA_OK) return sh;
@@ -349,7 +365,7 @@ void qlora_nf4_codebook(float out[16]) {
 }
 
 qlora_status qlora_codebook(int32_t code, float out[16]) {
-  const Nf4Params* P = code_params_or_null(code);
+  const Nf4Params* P = code_params_or_null(code & ~QLORA_DQ_CENTRED_FP8);
   if (!P || !out) return QLORA_ERR_INVALID_ARG;
   std::memcpy(out, P->q, sizeof(P->q));
   return QLORA_OK;

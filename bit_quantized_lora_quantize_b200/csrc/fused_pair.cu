@@ -456,9 +456,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const WaitCtx ctx{abort_flag, args.status, 23, args.wait_ns};
       const int grp = (warp - 4) >> 2;          // 0: even stages, 1: odd stages
       const int d = (threadIdx.x - 128) & 127;  // 0..127
-      lvl2[threadIdx.x - 128] = level2_value(threadIdx.x - 128);
+      lvl2[threadIdx.x - 128] = level2_value_for(threadIdx.x - 128, args.nf4.centred);
       asm volatile("bar.sync 1, 256;" ::: "memory");
       const int64_t blocks_per_row = args.w_cols / 64;
+      const float mu = centred_mu(args.absmax_scale, (args.w_rows * blocks_per_row + 255) / 256, args.nf4.centred);
       if (runit || tunit) {
         // Rank and tail units read no weight.  In the input gradient the
         // rank units' idle decoder threads write the bf16 pair of the saved
@@ -525,7 +526,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint4 v0 = *reinterpret_cast<const uint4*>(src + ((0 ^ sw) << 4));
             const uint4 v1 = *reinterpret_cast<const uint4*>(src + ((1 ^ sw) << 4));
             const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-            const Nf4Lut lut = make_lut(args.nf4, __fmul_rn(lvl2[q2], c1));
+            const Nf4Lut lut = make_lut(args.nf4, __fadd_rn(__fmul_rn(lvl2[q2], c1), mu));
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
               uint32_t o[4];
@@ -584,7 +585,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint4 v1 = *reinterpret_cast<const uint4*>(row + (((2 * j + 1) ^ sw) << 4));
             const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
             if (abs_tma) q2 = sAbs[s * 1024 + nl * 16 + abs_col];
-            const Nf4Lut lut = make_lut(args.nf4, __fmul_rn(lvl2[q2], c1));
+            const Nf4Lut lut = make_lut(args.nf4, __fadd_rn(__fmul_rn(lvl2[q2], c1), mu));
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
               uint32_t o[4];

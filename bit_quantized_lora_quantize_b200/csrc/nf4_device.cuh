@@ -28,6 +28,7 @@ namespace qlora {
 struct Nf4Params {
   float q[16];       // NF4 levels, ascending, float32
   double bnd[15];    // boundary B_j in x / c_b between code j and code j + 1
+  int centred;       // constants coded as E4M3 of (c_b - mu), see block_constant
 };
 
 // fp32(k / 255): level k of the 8-bit code of the absmax constants.
@@ -97,9 +98,30 @@ __device__ __forceinline__ void decode8(const Nf4Lut& L, uint32_t w, uint32_t (&
   out[3] = prmt(lo, hi, 0x6273);
 }
 
-// a' = fp32(fp32(k / 255) * c1)
-__device__ __forceinline__ float block_constant(uint32_t code2, float c1) {
-  return __fmul_rn(level2_value(code2), c1);
+// Value of an 8-bit E4M3 code (1 sign, 4 exponent bits with bias 7, 3
+// mantissa bits; subnormals at exponent 0).  Exact in float32.
+__device__ __forceinline__ float e4m3_value(uint32_t k) {
+  const uint32_t e = (k >> 3) & 15u, m = k & 7u;
+  const float v = e == 0 ? static_cast<float>(m) * 0.001953125f  // m * 2^-9
+                         : __uint_as_float(((e + 120u) << 23) | (m << 20));
+  return (k & 0x80u) ? -v : v;
+}
+
+// Level k of the 8-bit constant code: k / 255 (unsigned linear) or the
+// E4M3 value (mean-centred 8-bit float scheme).
+__device__ __forceinline__ float level2_value_for(uint32_t k, int centred) {
+  return centred ? e4m3_value(k) : level2_value(k);
+}
+
+// a' = fp32(fp32(level(k) * c1) + mu), with mu = 0 for the linear scheme
+// (adding +0 to a non-negative product leaves its bits unchanged).
+__device__ __forceinline__ float block_constant(uint32_t code2, float c1, int centred, float mu) {
+  return __fadd_rn(__fmul_rn(level2_value_for(code2, centred), c1), mu);
+}
+
+// mu of the mean-centred scheme: stored after the NB2 group scales.
+__device__ __forceinline__ float centred_mu(const float* absmax_scale, int64_t nb2, int centred) {
+  return centred ? __ldg(absmax_scale + nb2) : 0.0f;
 }
 
 // ------------------------------------------------------------------ encode

@@ -60,6 +60,106 @@ constexpr int kFastExpLo = 6;
 // qlora_check_status reports and clears it.
 __device__ int g_codec_status;
 
+// ---------------------------------------------------------------- mean-centred scheme
+// The mean mu of a tensor's block absmaxes is exact: every absmax c_b is a
+// bf16 value mant * 2^(e - 134) (e the biased exponent, at least 1; mant
+// 8 bits), so per-exponent integer sums of mant are exact and independent of
+// order.  One kernel accumulates them, a second rounds their mean once to
+// float32 with integer arithmetic, and the quantization kernel reads it.
+// The sums live in this library's device array (cleared before each use):
+// centred quantizations on one device must not overlap on the GPU.
+__device__ unsigned long long g_mean_bins[256];
+
+__global__ void __launch_bounds__(256) absmax_bins_kernel(const uint16_t* __restrict__ W, int64_t numel,
+                                                          unsigned long long* __restrict__ bins) {
+  __shared__ unsigned long long sb[256];
+  sb[threadIdx.x] = 0;
+  __syncthreads();
+  const int64_t nb = (numel + kBlock - 1) / kBlock;
+  const int64_t full = numel / kBlock;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; b < nb; b += stride) {
+    uint32_t mx = 0;  // |x| as bf16 bits, two halves: magnitudes order like unsigned integers
+    if (b < full) {
+      const uint4* p = reinterpret_cast<const uint4*>(W + b * kBlock);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint4 v = __ldg(p + i);
+        mx = __vmaxu2(mx, v.x & 0x7FFF7FFFu);
+        mx = __vmaxu2(mx, v.y & 0x7FFF7FFFu);
+        mx = __vmaxu2(mx, v.z & 0x7FFF7FFFu);
+        mx = __vmaxu2(mx, v.w & 0x7FFF7FFFu);
+      }
+    } else {
+      for (int64_t i = b * kBlock; i < numel; ++i) mx = __vmaxu2(mx, static_cast<uint32_t>(W[i]) & 0x7FFFu);
+    }
+    const uint32_t m = max(mx & 0xFFFFu, mx >> 16);
+    const uint32_t e = m >> 7, f = m & 127u;
+    if (m != 0) atomicAdd(&sb[e > 0 ? e : 1], static_cast<unsigned long long>(e > 0 ? 128u + f : f));
+  }
+  __syncthreads();
+  if (sb[threadIdx.x] != 0) atomicAdd(&bins[threadIdx.x], sb[threadIdx.x]);
+}
+
+// mu = fp32(sum / nb), round to nearest even, from the per-exponent sums
+// (one thread).  The sum scaled by 2^165 is an integer of at most 12 32-bit
+// limbs; long division by nb (< 2^32) and rounding at the float32 quantum.
+__global__ void centred_mean_kernel(const unsigned long long* __restrict__ bins, int64_t nb, float* __restrict__ mu) {
+  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  constexpr int kLimbs = 12;
+  uint32_t L[kLimbs] = {};
+  for (int e = 1; e < 256; ++e) {
+    const unsigned long long v = bins[e];
+    if (!v) continue;
+    const int sh = e - 1 + 32;  // mant * 2^(e - 134) * 2^165 = mant * 2^(e - 1 + 32)
+    const int li = sh >> 5, bo = sh & 31;
+    const unsigned long long lo = v << bo;
+    const unsigned long long hi = bo ? (v >> (64 - bo)) : 0ull;
+    const uint32_t add[3] = {static_cast<uint32_t>(lo), static_cast<uint32_t>(lo >> 32), static_cast<uint32_t>(hi)};
+    unsigned long long carry = 0;
+    for (int i = li; i < kLimbs; ++i) {
+      const unsigned long long t = static_cast<unsigned long long>(L[i]) + (i - li < 3 ? add[i - li] : 0u) + carry;
+      L[i] = static_cast<uint32_t>(t);
+      carry = t >> 32;
+      if (i - li >= 2 && carry == 0) break;
+    }
+  }
+  const unsigned long long d = static_cast<unsigned long long>(nb);
+  uint32_t Q[kLimbs];
+  unsigned long long rem = 0;
+  for (int i = kLimbs - 1; i >= 0; --i) {
+    const unsigned long long cur = (rem << 32) | L[i];
+    Q[i] = static_cast<uint32_t>(cur / d);
+    rem = cur % d;
+  }
+  int h = -1;  // highest set bit of Q
+  for (int i = kLimbs - 1; i >= 0 && h < 0; --i)
+    if (Q[i]) h = 32 * i + 31 - __clz(Q[i]);
+  if (h < 0) {  // below 2^-165: rounds to zero
+    *mu = 0.0f;
+    return;
+  }
+  const int shift = max(h - 23, 16);  // float32 quantum 2^(shift - 165), at least 2^-149
+  auto bit = [&](int pos) -> uint32_t { return pos < 0 ? 0u : (Q[pos >> 5] >> (pos & 31)) & 1u; };
+  uint32_t mant = 0;
+  for (int i = 23; i >= 0; --i) mant = (mant << 1) | bit(shift + i);
+  const uint32_t half = bit(shift - 1);
+  bool sticky = rem != 0;
+  for (int pos = shift - 2; pos >= 0 && !sticky; --pos) sticky = bit(pos) != 0;
+  if (half && (sticky || (mant & 1u))) ++mant;
+  const int ex = shift - 165;
+  const float p2 = ex >= -126 ? __uint_as_float(static_cast<uint32_t>(ex + 127) << 23) : __uint_as_float(1u << (ex + 149));
+  *mu = __fmul_rn(static_cast<float>(mant), p2);  // exact
+}
+
+// Nearest E4M3 code of v, ties to even, saturating; the sign of a negative
+// value is kept even when it rounds to zero.
+__device__ __forceinline__ uint32_t e4m3_code(float v) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(v));
+  return (static_cast<uint32_t>(r) & 0xFFu) | (v < 0.0f ? 0x80u : 0u);
+}
+
 __global__ void __launch_bounds__(kThreads, 3)
     quantize_nf4_kernel(const __grid_constant__ CUtensorMap tmW, const uint16_t* __restrict__ W, int64_t numel,
                         uint8_t* __restrict__ codes, uint8_t* __restrict__ absmax_q,
@@ -79,6 +179,7 @@ __global__ void __launch_bounds__(kThreads, 3)
   const int64_t nb = (numel + kBlock - 1) / kBlock;
   const int64_t nbytes = (numel + 1) / 2;
   const bool ragged_tail = (numel % kBlock) != 0;  // last group staged with plain loads
+  const float mu = centred_mu(absmax_scale, groups, P.centred);  // written by the mean kernel
 
   lvl2[tid] = static_cast<double>(level2_value(tid));
   for (int i = tid; i < 128 * 16; i += kThreads) {
@@ -156,9 +257,11 @@ __global__ void __launch_bounds__(kThreads, 3)
       mx = __hmax2(mx, *reinterpret_cast<__nv_bfloat162*>(&a));
     }
     const float c = fmaxf(__low2float(mx), __high2float(mx));
+    const int64_t blk = g * kGroup + tid;
+    const float dcen = __fsub_rn(c, mu);  // centred scheme: c_b - mu
 
-    // Group maximum c1.
-    float m = c;
+    // Group maximum c1 (of c_b, or of |c_b - mu| over the blocks present).
+    float m = P.centred ? (blk < nb ? fabsf(dcen) : 0.0f) : c;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
     if ((tid & 31) == 0) warp_max[tid >> 5] = m;
@@ -167,11 +270,14 @@ __global__ void __launch_bounds__(kThreads, 3)
 #pragma unroll
     for (int w = 1; w < kThreads / 32; ++w) c1 = fmaxf(c1, warp_max[w]);
 
-    const int64_t blk = g * kGroup + tid;
+    const float sg = __fdiv_rn(c1, 448.0f);  // centred scheme: group scale
     if (blk < nb) {
       // 8-bit code of c / c1: nearest fp32(k / 255), ties to the lower k.
+      // Centred scheme: E4M3 code of (c - mu) / sg.
       uint32_t code2 = 0;
-      if (c1 > 0.0f) {
+      if (P.centred) {
+        if (sg > 0.0f) code2 = e4m3_code(__fdiv_rn(dcen, sg));
+      } else if (c1 > 0.0f) {
         const float n2 = __fdiv_rn(c, c1);
         int k0 = __float2int_rn(n2 * 255.0f);
         k0 = max(2, min(253, k0));
@@ -188,7 +294,7 @@ __global__ void __launch_bounds__(kThreads, 3)
       }
       absmax_q[blk] = static_cast<uint8_t>(code2);
     }
-    if (tid == 0) absmax_scale[g] = c1;
+    if (tid == 0) absmax_scale[g] = P.centred ? sg : c1;
 
     // 4-bit codes of the block.
     Nf4Thresholds T;
@@ -240,7 +346,8 @@ __global__ void __launch_bounds__(kThreads) dequantize_nf4_kernel(const uint8_t*
   const bool full = base + kGroupElems <= numel;
 
   if (blk < nb) {
-    const float a = block_constant(absmax_q[blk], absmax_scale[blockIdx.x]);
+    const float mu = centred_mu(absmax_scale, (nb + kGroup - 1) / kGroup, P.centred);
+    const float a = block_constant(absmax_q[blk], absmax_scale[blockIdx.x], P.centred, mu);
     const Nf4Lut L = make_lut(P, a);
     const int64_t byte0 = blk * (kBlock / 2);
     uint32_t w[8];
@@ -302,6 +409,19 @@ cudaError_t launch_quantize_nf4(const uint16_t* W, int64_t numel, uint8_t* codes
   }
   cudaError_t e = cudaFuncSetAttribute(quantize_nf4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kQuantSmem);
   if (e != cudaSuccess) return e;
+  if (P.centred) {
+    // The exact mean of the block absmaxes first (two small kernels).
+    unsigned long long* bins = nullptr;
+    e = cudaGetSymbolAddress(reinterpret_cast<void**>(&bins), g_mean_bins);
+    if (e == cudaSuccess) e = cudaMemsetAsync(bins, 0, sizeof(unsigned long long) * 256, stream);
+    if (e != cudaSuccess) return e;
+    const int64_t nb = (numel + kBlock - 1) / kBlock;
+    const int64_t bgrid = std::min<int64_t>((nb + 255) / 256, static_cast<int64_t>(sm_count) * 8);
+    absmax_bins_kernel<<<static_cast<unsigned>(std::max<int64_t>(1, bgrid)), 256, 0, stream>>>(W, numel, bins);
+    centred_mean_kernel<<<1, 32, 0, stream>>>(bins, nb, absmax_scale + groups);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   const int64_t grid = std::min<int64_t>(groups, static_cast<int64_t>(sm_count) * 3);
   quantize_nf4_kernel<<<static_cast<unsigned>(grid), kThreads, kQuantSmem, stream>>>(map, W, numel, codes, absmax_q,
                                                                                       absmax_scale, P, wait_limit_ns());

@@ -277,7 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     fence_mbarrier_init();
   }
-  if (threadIdx.x < 256) lvl2[threadIdx.x] = level2_value(threadIdx.x);
+  if (threadIdx.x < 256) lvl2[threadIdx.x] = level2_value_for(threadIdx.x, args.nf4.centred);
   for (int i = threadIdx.x; i < 256 * 16; i += kThreads) {
     const int b = i >> 4;  // code byte: high nibble = first element
     pair_tab[i] = make_float2(args.nf4.q[b >> 4], args.nf4.q[b & 15]);
@@ -619,6 +619,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         c1 = __ldg(args.absmax_scale + (blk >> 8));
       }
     };
+    const float mu = centred_mu(args.absmax_scale, (static_cast<int64_t>(args.N) * KB + 255) / 256, args.nf4.centred);
     Cursor cur = cursor_at(grp);
     Cursor pre = cur;
     uint32_t pq[kPrefetch];
@@ -635,7 +636,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; i < kPrefetch; ++i) {
         if (!run) continue;
         const int jm = static_cast<int>(cur.j);
-        const float amax = __fmul_rn(lvl2[pq[i]], pc[i]);  // 0 for rows past N
+        // 0 for rows past N (mu for the centred scheme: those rows are never stored)
+        const float amax = __fadd_rn(__fmul_rn(lvl2[pq[i]], pc[i]), mu);
         fetch(pre, pq[i], pc[i]);
         advance(pre);
         const int s = jm % S;

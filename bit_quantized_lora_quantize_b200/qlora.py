@@ -18,8 +18,10 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libqlora.so")
 
 QLORA_OK = 0
-# 4-bit codes of the packed format (qlora_code in include/qlora.h).
+# 4-bit codes of the packed format (qlora_code in include/qlora.h) and the
+# schemes of the 8-bit constants (QLORA_DQ_CENTRED_FP8 for "centred_fp8").
 CODES = {"nf4": 0, "fp4": 1, "int4": 2}
+DQ = {"linear8": 0, "centred_fp8": 0x100}
 STATUS_NAMES = {0: "QLORA_OK", 1: "QLORA_ERR_INVALID_ARG", 2: "QLORA_ERR_ALIGNMENT", 3: "QLORA_ERR_UNSUPPORTED",
                 4: "QLORA_ERR_WORKSPACE", 5: "QLORA_ERR_CUDA", 6: "QLORA_ERR_TIMEOUT"}
 
@@ -125,6 +127,11 @@ class PackedNF4:
     absmax_scale: torch.Tensor  # float32 [NB2]
     shape: tuple
     code: str = "nf4"
+    dq: str = "linear8"
+
+    @property
+    def code_value(self) -> int:
+        return CODES[self.code] | DQ[self.dq]
 
     @property
     def numel(self) -> int:
@@ -151,32 +158,34 @@ def qlora_codebook(code: str = "nf4") -> list:
     return list(buf)
 
 
-def qlora_quantize_nf4(W: torch.Tensor, out: PackedNF4 = None, code: str = "nf4") -> PackedNF4:
+def qlora_quantize_nf4(W: torch.Tensor, out: PackedNF4 = None, code: str = "nf4", dq: str = "linear8") -> PackedNF4:
     """Quantize a bf16 CUDA tensor (any shape, flattened row-major) with the
-    NF4 levels (or ``code`` = "fp4" / "int4").  `out`, if given, is a
-    PackedNF4 of the same element count whose buffers are overwritten."""
+    NF4 levels (or ``code`` = "fp4" / "int4") and the linear 8-bit constants
+    (or ``dq`` = "centred_fp8").  `out`, if given, is a PackedNF4 of the same
+    element count whose buffers are overwritten."""
     _require_cuda(W)
     if W.dtype != torch.bfloat16:
         raise ValueError("W must be bfloat16")
     n = W.numel()
     nc, nb, nb2 = packed_sizes(n)
+    nsc = nb2 + (1 if dq == "centred_fp8" else 0)  # the centred scheme stores its mean last
     dev = W.device
     if out is None:
         codes = torch.empty(max(nc, 16), dtype=torch.uint8, device=dev)[:nc]
         aq = torch.empty(nb, dtype=torch.uint8, device=dev)
-        sc = torch.empty(nb2, dtype=torch.float32, device=dev)
+        sc = torch.empty(nsc, dtype=torch.float32, device=dev)
     else:
         codes, aq, sc = out.codes, out.absmax_q, out.absmax_scale
-        if (codes.numel(), aq.numel(), sc.numel()) != (nc, nb, nb2):
+        if (codes.numel(), aq.numel(), sc.numel()) != (nc, nb, nsc):
             raise ValueError("out does not hold a weight of this size")
         _require_cuda(codes, aq, sc)
-    if code == "nf4":
+    if code == "nf4" and dq == "linear8":
         _check("qlora_quantize_nf4", lib().qlora_quantize_nf4(_ptr(W), n, _ptr(codes), _ptr(aq), _ptr(sc),
                                                               _stream()))
     else:
-        _check("qlora_quantize_4bit", lib().qlora_quantize_4bit(_ptr(W), n, CODES[code], _ptr(codes), _ptr(aq),
-                                                                _ptr(sc), _stream()))
-    return PackedNF4(codes, aq, sc, tuple(W.shape), code)
+        _check("qlora_quantize_4bit", lib().qlora_quantize_4bit(_ptr(W), n, CODES[code] | DQ[dq], _ptr(codes),
+                                                                _ptr(aq), _ptr(sc), _stream()))
+    return PackedNF4(codes, aq, sc, tuple(W.shape), code, dq)
 
 
 def qlora_dequantize_nf4(p: PackedNF4, out: torch.Tensor = None) -> torch.Tensor:
@@ -185,12 +194,12 @@ def qlora_dequantize_nf4(p: PackedNF4, out: torch.Tensor = None) -> torch.Tensor
         out = torch.empty(p.shape, dtype=torch.bfloat16, device=p.codes.device)
     elif out.dtype != torch.bfloat16 or out.numel() != p.numel or not out.is_contiguous():
         raise ValueError("out must be a contiguous bf16 tensor of the weight's size")
-    if p.code == "nf4":
+    if p.code_value == 0:
         _check("qlora_dequantize_nf4", lib().qlora_dequantize_nf4(_ptr(p.codes), _ptr(p.absmax_q),
                                                                   _ptr(p.absmax_scale), p.numel, _ptr(out), _stream()))
     else:
         _check("qlora_dequantize_4bit", lib().qlora_dequantize_4bit(_ptr(p.codes), _ptr(p.absmax_q),
-                                                                    _ptr(p.absmax_scale), p.numel, CODES[p.code],
+                                                                    _ptr(p.absmax_scale), p.numel, p.code_value,
                                                                     _ptr(out), _stream()))
     return out
 
@@ -221,13 +230,13 @@ def qlora_linear_fwd(X: torch.Tensor, W: PackedNF4, A: torch.Tensor, B: torch.Te
         Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
     if T_save is None:
         T_save = torch.empty(M, r, dtype=torch.float32, device=dev)
-    if W.code == "nf4":
+    if W.code_value == 0:
         _check("qlora_linear_fwd", lib().qlora_linear_fwd(
             _ptr(X), M, K, N, _ptr(W.codes), _ptr(W.absmax_q), _ptr(W.absmax_scale), _ptr(A), _ptr(B), r,
             float(scale), _ptr(Y), _ptr(T_save), _ptr(workspace), workspace.numel(), _stream()))
     else:
         _check("qlora_linear_fwd_4bit", lib().qlora_linear_fwd_4bit(
-            _ptr(X), M, K, N, _ptr(W.codes), _ptr(W.absmax_q), _ptr(W.absmax_scale), CODES[W.code], _ptr(A),
+            _ptr(X), M, K, N, _ptr(W.codes), _ptr(W.absmax_q), _ptr(W.absmax_scale), W.code_value, _ptr(A),
             _ptr(B), r, float(scale), _ptr(Y), _ptr(T_save), _ptr(workspace), workspace.numel(), _stream()))
     return Y, T_save
 
@@ -236,8 +245,8 @@ def qlora_linear_fwd_noalloc(X: torch.Tensor, W: PackedNF4, A: torch.Tensor, B: 
                              Y: torch.Tensor, T_save: torch.Tensor):
     """Forward into caller-provided Y and T_save with no workspace: the
     library takes its scratch from a fixed device array (see include/qlora.h)."""
-    if W.code != "nf4":
-        raise ValueError("the allocation-free forward takes NF4 weights only")
+    if W.code_value != 0:
+        raise ValueError("the allocation-free forward takes NF4 weights with linear 8-bit constants only")
     M, K = X.shape
     N = W.shape[0]
     r = A.shape[1]
@@ -265,7 +274,7 @@ def qlora_linear_bwd(dY: torch.Tensor, X: torch.Tensor, T_save: torch.Tensor, W:
         dA = torch.empty(K, r, dtype=torch.float32, device=dev)
     if dB is None:
         dB = torch.empty(r, N, dtype=torch.float32, device=dev)
-    if W.code == "nf4":
+    if W.code_value == 0:
         _check("qlora_linear_bwd", lib().qlora_linear_bwd(
             _ptr(dY), _ptr(X), _ptr(T_save), M, K, N, _ptr(W.codes), _ptr(W.absmax_q), _ptr(W.absmax_scale),
             _ptr(A), _ptr(B), r, float(scale), _ptr(dX), _ptr(dA), _ptr(dB), _ptr(workspace), workspace.numel(),
@@ -273,7 +282,7 @@ def qlora_linear_bwd(dY: torch.Tensor, X: torch.Tensor, T_save: torch.Tensor, W:
     else:
         _check("qlora_linear_bwd_4bit", lib().qlora_linear_bwd_4bit(
             _ptr(dY), _ptr(X), _ptr(T_save), M, K, N, _ptr(W.codes), _ptr(W.absmax_q), _ptr(W.absmax_scale),
-            CODES[W.code], _ptr(A), _ptr(B), r, float(scale), _ptr(dX), _ptr(dA), _ptr(dB), _ptr(workspace),
+            W.code_value, _ptr(A), _ptr(B), r, float(scale), _ptr(dX), _ptr(dA), _ptr(dB), _ptr(workspace),
             workspace.numel(), _stream()))
     return dX, dA, dB
 

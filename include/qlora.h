@@ -88,6 +88,25 @@ typedef enum {
 typedef enum { QLORA_CODE_NF4 = 0, QLORA_CODE_FP4 = 1, QLORA_CODE_INT4 = 2 } qlora_code;
 
 /*
+ * Second reading of "2. Double Quantization" (the pages say only that the
+ * constants are quantized; this is the original QLoRA paper's variant, not
+ * printed on the pages).  OR-ed into a qlora_code, it codes the constants as
+ * 8-bit floats after removing their mean:
+ *   mu   = fp32(exact mean of every block absmax c_b of the tensor)
+ *   s_g  = fp32(max |fp32(c_b - mu)| over the 256-group / 448)
+ *   k_b  = E4M3 code (sign, 4 exponent bits with bias 7, 3 mantissa bits)
+ *          nearest to fp32(fp32(c_b - mu) / s_g), ties to the even code,
+ *          saturating at +-448, -0 kept; 0 when s_g = 0
+ *   a'   = fp32(fp32(E4M3(k_b) * s_g) + mu)
+ * absmax_q holds k_b; absmax_scale holds NB2 + 1 floats: s_g per group,
+ * then mu.  The 4-bit codes still use the true c_b.  Quantization runs three
+ * kernels (exact per-exponent sums of the absmaxes in a device array of this
+ * library, their mean, then the codes): centred quantizations on one device
+ * must not overlap on the GPU, and numel is limited to 2^38.
+ */
+#define QLORA_DQ_CENTRED_FP8 0x100
+
+/*
  * Blockwise NF4 quantization with double-quantized constants.
  * "AI Glossary: QLoRA", second paragraph; "1. 4-bit NormalFloat (NF4)" and
  * "2. Double Quantization" in "QLoRA: Fine-Tuning 65-Billion Parameter
@@ -104,9 +123,9 @@ typedef enum { QLORA_CODE_NF4 = 0, QLORA_CODE_FP4 = 1, QLORA_CODE_INT4 = 2 } qlo
 QLORA_API qlora_status qlora_quantize_nf4(const uint16_t* W, int64_t numel, uint8_t* codes, uint8_t* absmax_q,
                                 float* absmax_scale, void* stream);
 
-/* The same quantization with the levels of `code` (a qlora_code; any other
- * value returns QLORA_ERR_INVALID_ARG).  qlora_quantize_nf4 is this call
- * with QLORA_CODE_NF4. */
+/* The same quantization with the levels of `code` (a qlora_code, optionally
+ * OR QLORA_DQ_CENTRED_FP8; any other value returns QLORA_ERR_INVALID_ARG).
+ * qlora_quantize_nf4 is this call with QLORA_CODE_NF4. */
 QLORA_API qlora_status qlora_quantize_4bit(const uint16_t* W, int64_t numel, int32_t code, uint8_t* codes,
                                            uint8_t* absmax_q, float* absmax_scale, void* stream);
 
