@@ -32,23 +32,43 @@ constexpr size_t kStatusBytes = 256;
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// The kernels take ranks that are multiples of 8 (the adapter rows are copied
+// by TMA, whose row strides are multiples of 16 bytes); other ranks run with
+// the adapter padded by zero columns to r8 in the workspace.
+int rank8(int r) { return (r + 7) / 8 * 8; }
+
+// The weight-streaming forward holds rank indices in one 128-row MMA tile.
+bool small_m_path(int64_t M, int r) { return M <= kSmallMMax && rank8(r) <= 128; }
+
 // Workspace: [status word (256 B)][counters of the forward and input-gradient
-// GEMMs][T pair: bf16 M x 2rp][U pair: bf16 M x 2rp] and, when
-// M <= kSmallMMax, [small-M counters and partial tiles].
+// GEMMs][T pair: bf16 M x 2rp][U pair: bf16 M x 2rp]; when the small-M
+// forward runs, [its counters and partial tiles]; when r % 8 != 0, [A, B, T,
+// dA, dB padded to r8].
 struct WsLayout {
-  size_t cf_off, cd_off, t_off, u_off, sm_off, total;
+  size_t cf_off, cd_off, t_off, u_off, sm_off, pad_off;
+  size_t pa_off, pb_off, pt_off, pda_off, pdb_off, total;
 };
 
 WsLayout ws_layout(int64_t M, int64_t K, int64_t N, int r) {
   WsLayout w{};
-  const size_t pair_bytes = round_up(static_cast<size_t>(M) * 2 * lora_pad(r) * 2, 256);
+  const int r8 = rank8(r);
+  const size_t pair_bytes = round_up(static_cast<size_t>(M) * 2 * lora_pad(r8) * 2, 256);
   const size_t ctr_bytes = round_up(static_cast<size_t>(fused_ctr_ints(M)) * 4, 256);
   w.cf_off = kStatusBytes;
   w.cd_off = w.cf_off + ctr_bytes;
   w.t_off = w.cd_off + ctr_bytes;
   w.u_off = w.t_off + pair_bytes;
   w.sm_off = w.u_off + pair_bytes;
-  w.total = w.sm_off + (M <= kSmallMMax ? round_up(small_m_workspace_bytes(M, N, r), 256) : 0);
+  w.pad_off = w.sm_off + (small_m_path(M, r) ? round_up(small_m_workspace_bytes(M, N, r8), 256) : 0);
+  size_t o = w.pad_off;
+  if (r8 != r) {
+    w.pa_off = o; o += round_up(static_cast<size_t>(K) * r8 * 2, 256);
+    w.pb_off = o; o += round_up(static_cast<size_t>(r8) * N * 2, 256);
+    w.pt_off = o; o += round_up(static_cast<size_t>(M) * r8 * 4, 256);
+    w.pda_off = o; o += round_up(static_cast<size_t>(K) * r8 * 4, 256);
+    w.pdb_off = o; o += round_up(static_cast<size_t>(r8) * N * 4, 256);
+  }
+  w.total = o;
   return w;
 }
 
@@ -114,7 +134,7 @@ qlora_status cuda_fail(cudaError_t e) {
 qlora_status check_linear_shape(int64_t M, int64_t K, int64_t N, int32_t r) {
   if (M <= 0 || K <= 0 || N <= 0 || r <= 0) return QLORA_ERR_INVALID_ARG;
   if (M >= (int64_t(1) << 31) || K >= (int64_t(1) << 31) || N >= (int64_t(1) << 31)) return QLORA_ERR_UNSUPPORTED;
-  if (K % 64 != 0 || N % 8 != 0 || r % 8 != 0 || r > 128) return QLORA_ERR_UNSUPPORTED;
+  if (K % 64 != 0 || N % 8 != 0 || r > 256) return QLORA_ERR_UNSUPPORTED;
   return QLORA_OK;
 }
 
@@ -227,23 +247,39 @@ qlora_status qlora_linear_fwd_4bit(const uint16_t* X, int64_t M, int64_t K, int6
   const Nf4Params& P = *Pc;
 
   uint16_t* Tpair = reinterpret_cast<uint16_t*>(ws + wl.t_off);
-
-  if (M <= kSmallMMax) {
+  const int r8 = rank8(r);
+  const uint16_t* Ak = A;
+  const uint16_t* Bk = B;
+  float* Tk = T_save;
+  if (r8 != r) {
+    // The adapter padded with zero columns (A) and rows (B) to r8; T comes
+    // back through a padded buffer.
+    uint16_t* Ap = reinterpret_cast<uint16_t*>(ws + wl.pa_off);
+    uint16_t* Bp = reinterpret_cast<uint16_t*>(ws + wl.pb_off);
+    cudaError_t e = launch_pad_copy(A, K, r, r, Ap, r8, r8, 2, st);
+    if (e == cudaSuccess) e = launch_pad_copy(B, r, N, N, Bp, N, N, 2, st, r8);
+    if (e != cudaSuccess) return cuda_fail(e);
+    Ak = Ap;
+    Bk = Bp;
+    Tk = reinterpret_cast<float*>(ws + wl.pt_off);
+  }
+  cudaError_t e;
+  if (small_m_path(M, r)) {
     // One launch: T, its pair and Y.
     ProfScope p0(st, "small_m_nf4_fwd", 1);
-    const cudaError_t e = launch_small_m_fwd(X, codes, absmax_q, absmax_scale, A, B, M, K, N, r, scale, Y, T_save,
-                                             Tpair, ws + wl.sm_off, status, P, st);
+    e = launch_small_m_fwd(X, codes, absmax_q, absmax_scale, Ak, Bk, M, K, N, r8, scale, Y, Tk, Tpair,
+                           ws + wl.sm_off, status, P, st);
     p0.done();
-    return e == cudaSuccess ? QLORA_OK : cuda_fail(e);
+  } else {
+    // One launch: T = s X A (T_save and its pair) in the kernel's first
+    // units, then the output tiles.
+    ProfScope p2(st, "fused_nf4_fwd", 1);
+    e = launch_fused_fwd(X, codes, absmax_q, absmax_scale, Tpair, Bk, M, K, N, r8, Y, status, P, st, Ak, Tk, scale,
+                         reinterpret_cast<int*>(ws + wl.cf_off));
+    p2.done();
   }
-  // One launch: T = s X A (T_save and its pair) in the kernel's first units,
-  // then the output tiles.
-  ProfScope p2(st, "fused_nf4_fwd", 1);
-  const cudaError_t e = launch_fused_fwd(X, codes, absmax_q, absmax_scale, Tpair, B, M, K, N, r, Y, status, P, st, A,
-                                         T_save, scale, reinterpret_cast<int*>(ws + wl.cf_off));
-  p2.done();
-  if (e != cudaSuccess) return cuda_fail(e);
-  return QLORA_OK;
+  if (e == cudaSuccess && r8 != r) e = launch_pad_copy(Tk, M, r8, r8, T_save, r, r, 4, st);
+  return e == cudaSuccess ? QLORA_OK : cuda_fail(e);
 }
 
 qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, int64_t K, int64_t N, const uint8_t* codes,
@@ -281,15 +317,39 @@ qlora_status qlora_linear_bwd_4bit(const uint16_t* dY, const uint16_t* X, const 
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   const Nf4Params& P = *Pc;
 
+  const int r8 = rank8(r);
+  const uint16_t* Ak = A;
+  const uint16_t* Bk = B;
+  const float* Tk = T_save;
+  float* dAk = dA;
+  float* dBk = dB;
+  cudaError_t e = cudaSuccess;
+  if (r8 != r) {
+    uint16_t* Ap = reinterpret_cast<uint16_t*>(ws + wl.pa_off);
+    uint16_t* Bp = reinterpret_cast<uint16_t*>(ws + wl.pb_off);
+    float* Tp = reinterpret_cast<float*>(ws + wl.pt_off);
+    e = launch_pad_copy(A, K, r, r, Ap, r8, r8, 2, st);
+    if (e == cudaSuccess) e = launch_pad_copy(B, r, N, N, Bp, N, N, 2, st, r8);
+    if (e == cudaSuccess) e = launch_pad_copy(T_save, M, r, r, Tp, r8, r8, 4, st);
+    if (e != cudaSuccess) return cuda_fail(e);
+    Ak = Ap;
+    Bk = Bp;
+    Tk = Tp;
+    dAk = reinterpret_cast<float*>(ws + wl.pda_off);
+    dBk = reinterpret_cast<float*>(ws + wl.pdb_off);
+  }
   // One launch: U = s dY B^T (and the bf16 pair of T) in the first units,
   // the dX tiles, and dA = X^T U and dB = T^T dY in units that fill the SMs
   // the last wave of tiles leaves idle.
   ProfScope p2(st, "fused_nf4_dx", 1);
-  const cudaError_t e = launch_fused_dx(dY, codes, absmax_q, absmax_scale, Upair, A, M, K, N, r, dX, status, P, st,
-                                        B, scale, reinterpret_cast<int*>(ws + wl.cd_off), X, T_save, Tpair, dA, dB);
+  e = launch_fused_dx(dY, codes, absmax_q, absmax_scale, Upair, Ak, M, K, N, r8, dX, status, P, st, Bk, scale,
+                      reinterpret_cast<int*>(ws + wl.cd_off), X, Tk, Tpair, dAk, dBk);
   p2.done();
-  if (e != cudaSuccess) return cuda_fail(e);
-  return QLORA_OK;
+  if (e == cudaSuccess && r8 != r) {
+    e = launch_pad_copy(dAk, K, r8, r8, dA, r, r, 4, st);
+    if (e == cudaSuccess) e = launch_pad_copy(dBk, r, N, N, dB, N, N, 4, st);
+  }
+  return e == cudaSuccess ? QLORA_OK : cuda_fail(e);
 }
 
 qlora_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, const float* T_save, int64_t M, int64_t K,

@@ -76,9 +76,11 @@ struct PairArgs {
   float scale;      // LoRA scale s, applied to the rank-r intermediate
   float* r_f32;     // float32 intermediate [rows x r] (forward T) or null
   uint16_t* r_pair; // bf16 pair of the intermediate, read by the LoRA stages
-  // Tail units (input gradient only): da_units of dA then dB ones.  The first
+  // Tail units (input gradient only): for each chunk of t_chunk adapter
+  // columns, da_units of dA then the dB ones (t_base per chunk).  The first
   // t_first go out after the first `early` tiles, the rest after all tiles.
-  int t_units, da_units, early, t_first;
+  int t_units, da_units, early, t_first, t_base, t_chunk;
+  int unit_cols;    // adapter columns per CTA of a rank unit (64 or 128)
   int nmb;          // 64-row blocks of M (reduction depth of a tail unit)
   float* dA;        // [K x r]
   float* dB;        // [r x N]
@@ -211,7 +213,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                       const __grid_constant__ TailMaps tm, const PairArgs args) {
   using L = PairSmem<MNB>;
   constexpr uint32_t kTmemCols = 512;  // two 128 x 256 fp32 accumulators
-  constexpr int kRankB = 64 * kDepth * 2;  // a rank unit's adapter tile per CTA and stage
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -307,8 +308,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int row0 = tile_m * kPairRows + static_cast<int>(rank) * 128;
         if (tunit) {
           // 64 tokens per stage: this CTA's 2 x 128 result rows of the
-          // activation (four 64-column boxes) and its rp columns of the pair.
-          const bool is_da = tj < args.da_units;
+          // activation (four 64-column boxes) and its t_chunk columns of the
+          // pair (the hi half in the leader, the lo half in the peer).
+          const int chunk = tj / args.t_base, tb = tj - chunk * args.t_base;
+          const bool is_da = tb < args.da_units;
           if (i == 0) {
             bool ok = true;
             for (int m = 0; m < args.r_units && ok; ++m) ok = wait_count(args.ctr + 2 + m, 2, ctx);
@@ -317,8 +320,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const CUtensorMap* am = is_da ? &tm.a_da : &tm.a_db;
           const CUtensorMap* bm = is_da ? &tm.b_da : &tm.b_db;
-          const int c0 = (is_da ? tj : tj - args.da_units) * kPairRows + static_cast<int>(rank) * 128;
-          const int nb = args.lora_mod / 64;
+          const int c0 = (is_da ? tb : tb - args.da_units) * kPairRows + static_cast<int>(rank) * 128;
+          const int nb = args.t_chunk / 64;
           if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * L::kA + 2 * nb * 8192);
 #pragma unroll
           for (int h = 0; h < 2; ++h)
@@ -326,22 +329,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int a = 0; a < 2; ++a)
               tma_load_2d_pair(am, full_leader, a_dst + h * 16384 + a * 8192, c0 + h * 256 + a * 64, i * kDepth);
           for (int b = 0; b < nb; ++b)
-            tma_load_2d_pair(bm, full_leader, b_dst + b * 8192, static_cast<int>(rank) * args.lora_mod + b * 64,
-                             i * kDepth);
+            tma_load_2d_pair(bm, full_leader, b_dst + b * 8192,
+                             static_cast<int>(rank) * args.lora_mod + chunk * args.t_chunk + b * 64, i * kDepth);
           ++issued;
           continue;
         }
         if (i < args.nkb) {
           const int kb = i;
-          if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * L::kA + (runit ? 2 * kRankB : 0));
+          if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * L::kA + (runit ? 2 * args.unit_cols * kDepth * 2 : 0));
           tma_load_2d_pair(&tmA, full_leader, a_dst, kb * kDepth, row0);
           tma_load_2d_pair(&tmA, full_leader, a_dst + 16384, kb * kDepth, row0 + 256);
           if (runit) {
-            // This CTA's 64 adapter columns: forward A[K, r] rows of block kb
-            // (MN-major B operand), input gradient B[r, N] columns of block kb
-            // (K-major).  Columns past r read as zeros.
-            if (!MNB) tma_load_2d_pair(&tmR, full_leader, b_dst, static_cast<int>(rank) * 64, kb * kDepth);
-            else tma_load_2d_pair(&tmR, full_leader, b_dst, kb * kDepth, static_cast<int>(rank) * 64);
+            // This CTA's unit_cols adapter columns (64-wide boxes): forward
+            // A[K, r] rows of block kb (MN-major B operand), input gradient
+            // B[r, N] columns of block kb (K-major).  Columns past r read as
+            // zeros.
+            for (int b = 0; b < args.unit_cols / 64; ++b) {
+              const int col = static_cast<int>(rank) * args.unit_cols + b * 64;
+              if (!MNB) tma_load_2d_pair(&tmR, full_leader, b_dst + b * 8192, col, kb * kDepth);
+              else tma_load_2d_pair(&tmR, full_leader, b_dst + b * 8192, kb * kDepth, col);
+            }
             ++issued;
             continue;
           }
@@ -408,8 +415,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // M = 256 across the pair, N = 256 (each CTA supplies 128 columns of B).
       const uint32_t idesc_main = idesc_bf16_f32(256, 256, false, MNB);
       const uint32_t idesc_lora = idesc_bf16_f32(256, 256, false, !MNB);
-      const uint32_t idesc_unit = idesc_bf16_f32(256, 128, false, !MNB);
-      const uint32_t idesc_tail = idesc_bf16_f32(256, 2 * args.lora_mod, true, true);
+      const uint32_t idesc_unit = idesc_bf16_f32(256, 2 * args.unit_cols, false, !MNB);
+      const uint32_t idesc_tail = idesc_bf16_f32(256, 2 * args.t_chunk, true, true);
       const uint32_t d = tmem_acc + h * 256;
       bool ok = true;
       for (int i = 0; i < total && ok; ++i) {
@@ -654,23 +661,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       } else if (ok && tunit) {
-        // Result rows (k of dA, n of dB) in lanes; columns [0, rp) hold the
-        // product with the hi half of the pair, [rp, 2rp) with the lo half.
-        const int rp = args.lora_mod;
-        const bool is_da = tj < args.da_units;
-        const int rrow = (is_da ? tj : tj - args.da_units) * kPairRows + h * 256 + static_cast<int>(rank) * 128 +
+        // Result rows (k of dA, n of dB) in lanes; columns [0, rc) hold the
+        // product with the chunk's hi half of the pair, [rc, 2rc) with its lo
+        // half (rc = t_chunk adapter columns, chunk `chunk`).
+        const int rc = args.t_chunk;
+        const int chunk = tj / args.t_base, tb = tj - chunk * args.t_base;
+        const bool is_da = tb < args.da_units;
+        const int rrow = (is_da ? tb : tb - args.da_units) * kPairRows + h * 256 + static_cast<int>(rank) * 128 +
                          q * 32 + lane;
         const bool in = rrow < (is_da ? args.w_cols : args.w_rows);
 #pragma unroll 1
-        for (int cc = 0; cc < rp / 32; ++cc) {
+        for (int cc = 0; cc < rc / 32; ++cc) {
           uint32_t vh[32], vl[32];
           tmem_ld_32x32b_x32(t_row + cc * 32, vh);
-          tmem_ld_32x32b_x32(t_row + rp + cc * 32, vl);
+          tmem_ld_32x32b_x32(t_row + rc + cc * 32, vl);
           tmem_wait_ld();
           if (in) {
 #pragma unroll
             for (int e = 0; e < 32; e += 4) {
-              const int j = cc * 32 + e;
+              const int j = chunk * rc + cc * 32 + e;
               if (j < args.r) {
                 const float4 o = make_float4(__fadd_rn(__uint_as_float(vh[e]), __uint_as_float(vl[e])),
                                              __fadd_rn(__uint_as_float(vh[e + 1]), __uint_as_float(vl[e + 1])),
@@ -807,6 +816,9 @@ void plan_units(PairArgs& args, int64_t M, int64_t cols, int64_t depth, int r, f
   args.r_f32 = r_f32;
   args.r_pair = r_pair;
   args.early = tiles_m * tiles_n;
+  const int rp = lora_pad(r);
+  args.unit_cols = rp <= 128 ? 64 : 128;               // N = 2 * unit_cols <= 256 across the pair
+  args.t_chunk = rp <= 128 ? rp : (rp % 128 == 0 ? 128 : 64);
 }
 
 // CTA pairs resident at once (one 1-CTA-per-SM pair per two SMs).
@@ -901,7 +913,8 @@ cudaError_t launch_fused_dx(const uint16_t* dY, const uint8_t* codes, const uint
                      CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
     args.da_units = static_cast<int>((K + kPairRows - 1) / kPairRows);
-    args.t_units = args.da_units + static_cast<int>((N + kPairRows - 1) / kPairRows);
+    args.t_base = args.da_units + static_cast<int>((N + kPairRows - 1) / kPairRows);
+    args.t_units = args.t_base * (rp / args.t_chunk);
     args.early = std::min(args.early, std::max(0, resident_pairs() - args.r_units));
     args.t_first = std::min(args.t_units, args.r_units);
     args.units += args.t_units;

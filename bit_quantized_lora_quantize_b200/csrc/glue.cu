@@ -1,5 +1,6 @@
 // SiLU gate between the linears of a gated MLP (LLaMA's feed-forward block):
-// H = silu(G) * U and its backward.  This is glue between LoRA linears, not a
+// H = silu(G) * U and its backward; and the copy that pads the adapter to a
+// multiple of 8 ranks.  This is glue between LoRA linears, not a
 // step of the QLoRA method; it exists so that a whole gated MLP runs on this
 // library's kernels.  Elementwise and HBM-bound: 16-byte vector loads and
 // stores, float32 arithmetic, one bf16 rounding per output.
@@ -94,7 +95,35 @@ int glue_grid(int64_t n8) {
   return static_cast<int>(std::max<int64_t>(1, std::min(want, cap)));
 }
 
+template <typename T>
+__global__ void __launch_bounds__(kGlueThreads) pad_copy_kernel(const T* __restrict__ src, int64_t rows,
+                                                                int64_t src_cols, int64_t src_ld, T* __restrict__ dst,
+                                                                int64_t dst_cols, int64_t dst_ld, int64_t dst_rows) {
+  const int64_t n = dst_rows * dst_cols;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += stride) {
+    const int64_t r = i / dst_cols, c = i - r * dst_cols;
+    dst[r * dst_ld + c] = (r < rows && c < src_cols) ? src[r * src_ld + c] : T(0);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_pad_copy(const void* src, int64_t rows, int64_t src_cols, int64_t src_ld, void* dst,
+                            int64_t dst_cols, int64_t dst_ld, int elem_bytes, cudaStream_t stream,
+                            int64_t dst_rows) {
+  if (dst_rows < 0) dst_rows = rows;
+  const int grid = glue_grid((dst_rows * dst_cols + 7) / 8);
+  if (elem_bytes == 2)
+    pad_copy_kernel<uint16_t><<<grid, kGlueThreads, 0, stream>>>(static_cast<const uint16_t*>(src), rows, src_cols,
+                                                                  src_ld, static_cast<uint16_t*>(dst), dst_cols,
+                                                                  dst_ld, dst_rows);
+  else
+    pad_copy_kernel<uint32_t><<<grid, kGlueThreads, 0, stream>>>(static_cast<const uint32_t*>(src), rows, src_cols,
+                                                                  src_ld, static_cast<uint32_t*>(dst), dst_cols,
+                                                                  dst_ld, dst_rows);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_silu_gate_fwd(const uint16_t* G, const uint16_t* U, uint16_t* H, int64_t n, cudaStream_t stream) {
   const int64_t n8 = n / 8;

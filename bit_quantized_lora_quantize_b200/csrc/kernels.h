@@ -82,6 +82,14 @@ cudaError_t launch_small_m_fwd(const uint16_t* X, const uint8_t* codes, const ui
                                int64_t K, int64_t N, int r, float scale, uint16_t* Y, float* T_save, uint16_t* Tpair,
                                void* scratch, int* status, const Nf4Params& P, cudaStream_t stream);
 
+// Copy a rows x src_cols matrix (row stride src_ld elements of elem_bytes,
+// 2 or 4) into dst (row stride dst_ld), filling columns [src_cols, dst_cols)
+// and rows [rows, dst_rows) with zeros (dst_rows = rows when omitted).  Used to
+// pad the adapter and its gradients to a multiple of 8 ranks.
+cudaError_t launch_pad_copy(const void* src, int64_t rows, int64_t src_cols, int64_t src_ld, void* dst,
+                            int64_t dst_cols, int64_t dst_ld, int elem_bytes, cudaStream_t stream,
+                            int64_t dst_rows = -1);
+
 // SiLU gate of a gated MLP (glue between linears): H = silu(G) * U and its
 // backward dG, dU, elementwise over n bf16 values.
 cudaError_t launch_silu_gate_fwd(const uint16_t* G, const uint16_t* U, uint16_t* H, int64_t n, cudaStream_t stream);

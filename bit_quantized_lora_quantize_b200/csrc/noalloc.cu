@@ -97,6 +97,7 @@ extern "C" qlora_status qlora_linear_fwd_noalloc(const uint16_t* X, int64_t M, i
   if (!(scale == scale) || scale - scale != 0.0f) return QLORA_ERR_INVALID_ARG;  // NaN or infinite
   const qlora_status sh = check_linear_shape(M, K, N, r);
   if (sh != QLORA_OK) return sh;
+  if (r % 8 != 0) return QLORA_ERR_UNSUPPORTED;  // no room for the padded adapter here
   if (!aligned16(X) || !aligned16(codes) || !aligned16(A) || !aligned16(B) || !aligned16(Y) || !aligned16(T_save) ||
       (reinterpret_cast<uintptr_t>(absmax_scale) & 3u))
     return QLORA_ERR_ALIGNMENT;

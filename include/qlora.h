@@ -167,8 +167,12 @@ QLORA_API qlora_status qlora_dequantize_4bit(const uint8_t* codes, const uint8_t
  *                 everything else is overwritten before it is read.  After
  *                 qlora_check_status reports QLORA_ERR_TIMEOUT, fill it with
  *                 zeros again before the next call.
- * Supported: K % 64 == 0, N % 8 == 0, r % 8 == 0 with 8 <= r <= 128,
- * M, N, K < 2^31.  Otherwise QLORA_ERR_UNSUPPORTED.
+ * Supported: K % 64 == 0, N % 8 == 0 (the weight's blocks and the row
+ * strides of Y, dY and B, which are copied by TMA, in 16-byte units),
+ * 1 <= r <= 256, M, N, K < 2^31.  Otherwise QLORA_ERR_UNSUPPORTED.  Ranks
+ * that are not multiples of 8 run with A, B, T_save, dA and dB padded with
+ * zeros to the next multiple of 8 inside the workspace (a few small copy
+ * kernels around the GEMM); ranks above 128 always take the pair GEMMs.
  * The forward is one kernel launch.  For M <= 128 its thread blocks wait
  * for one another (cooperative launch: all of them must be resident at
  * once); if the device cannot hold them next to other work the call returns
@@ -226,7 +230,9 @@ QLORA_API qlora_status qlora_linear_bwd_4bit(const uint16_t* dY, const uint16_t*
  * embedding that owns all device memory up front).  The QLoRA pages have no
  * counterpart to this call; it exists for those callers only.
  *   Same arguments, outputs and supported shapes as qlora_linear_fwd, minus
- *   workspace/ws_bytes; the results agree with qlora_linear_fwd to within
+ *   workspace/ws_bytes and ranks that are not multiples of 8
+ *   (QLORA_ERR_UNSUPPORTED: the padded adapter needs a workspace); the
+ *   results agree with qlora_linear_fwd to within
  *   float32 summation order: for every M this call runs the pair GEMM of the
  *   large-M forward, while qlora_linear_fwd takes the weight-streaming kernel
  *   for M <= 128.

@@ -96,8 +96,8 @@ def test_linear_fwd_validation(L):
     assert fwd(L, M=0) == 1
     assert fwd(L, K=100) == 3          # K % 64 != 0
     assert fwd(L, N=260) == 3          # N % 8 != 0
-    assert fwd(L, r=12) == 3           # r % 8 != 0
-    assert fwd(L, r=136) == 3          # r > 128
+    assert fwd(L, r=257) == 3          # r > 256
+    assert fwd(L, r=0) == 1
     assert fwd(L, X=FAKE + 8) == 2     # misaligned
     assert fwd(L, ws=None) == 4
     assert fwd(L, nws=16) == 4
@@ -124,6 +124,17 @@ def test_codec_validation(L):
     assert L.qlora_quantize_nf4(FAKE + 2, 64, FAKE, FAKE, FAKE, None) == 2
     assert L.qlora_dequantize_nf4(FAKE, FAKE, FAKE, -5, FAKE, None) == 1
     assert L.qlora_dequantize_nf4(FAKE, FAKE, FAKE + 2, 64, FAKE, None) == 2
+
+
+def test_any_rank_up_to_256_is_accepted(L):
+    """Ranks that are not multiples of 8 run with the adapter padded inside
+    the workspace, which is therefore larger; ranks above 128 take the pair
+    GEMMs for every M; 257 and above are unsupported."""
+    for r in (1, 4, 13, 64, 100, 136, 200, 256):
+        assert q.qlora_workspace_bytes(16, 256, 256, r) > 0
+        assert q.qlora_workspace_bytes(1000, 512, 384, r) > 0
+    assert q.qlora_workspace_bytes(16, 256, 256, 257) == 0
+    assert q.qlora_workspace_bytes(1000, 512, 384, 13) > q.qlora_workspace_bytes(1000, 512, 384, 16)
 
 
 def test_workspace_bytes(L):

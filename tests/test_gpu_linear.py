@@ -158,3 +158,16 @@ def test_attention_projection_full_size_sampled_rows():
     U = case.scale * (dY @ B.T)
     assert_close_rms(f64(g["dA"]), X.T @ U, "dA")
     assert_close_rms(f64(g["dB"]), case.scale * (X @ A).T @ dY, "dB")
+
+
+# Any rank 1 <= r <= 256: multiples of 8 up to 128 run as they are, others
+# with the adapter padded to a multiple of 8 in the workspace, and ranks above
+# 128 with the rank units taking 128 adapter columns per CTA and the dA / dB
+# units split into column chunks.  Large-M (pair GEMMs) and small-M shapes.
+@pytest.mark.parametrize("M,K,N,r", [(600, 512, 776, 4), (600, 512, 776, 200), (300, 320, 264, 1),
+                                     (700, 640, 392, 13), (520, 576, 520, 136), (600, 512, 256, 192),
+                                     (1100, 512, 640, 256), (16, 4096, 1024, 4), (16, 2048, 1000, 200),
+                                     (64, 1024, 512, 77), (1, 256, 256, 256)])
+def test_any_rank(M, K, N, r):
+    case = synthetic.linear_case(M, K, N, r, 0.5, seed=M + K + N + r)
+    check_full(case, run_gpu(case))
