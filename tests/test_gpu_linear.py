@@ -171,3 +171,17 @@ def test_attention_projection_full_size_sampled_rows():
 def test_any_rank(M, K, N, r):
     case = synthetic.linear_case(M, K, N, r, 0.5, seed=M + K + N + r)
     check_full(case, run_gpu(case))
+
+
+# One token (M = 1): ragged row counts and depths, every rank path.
+@pytest.mark.parametrize("K,N,r", [(64, 8, 8), (1024, 1000, 64), (16384, 136, 16), (4096, 4104, 5),
+                                   (8192, 1024, 256), (16448, 264, 64)])
+def test_single_token(K, N, r):
+    case = synthetic.linear_case(1, K, N, r, 0.5, seed=K + N + r)
+    check_full(case, run_gpu(case))
+
+
+def test_single_token_is_bit_reproducible():
+    case = synthetic.linear_case(1, 8192, 2056, 64, 0.25, seed=44)
+    g1, g2 = run_gpu(case), run_gpu(case)
+    assert torch.equal(g1["Y"], g2["Y"]) and torch.equal(g1["T"], g2["T"])
