@@ -714,6 +714,47 @@ def bench_attn(args, q, synthetic, dev, flush, peaks, local_rank):
     return res
 
 
+# ---------------------------------------------------------------- single small layer
+def bench_tiny(args, q, synthetic, dev, flush, iters=50):
+    """The small parity case (W 256 x 256, 16 tokens, r = 8, scale 2):
+    microseconds per quantize + forward + backward, each iteration after an
+    L2 flush.  Launch-bound: three launches per step."""
+    import torch
+    case = synthetic.tiny_case()
+    W = case.W.to(dev)
+    X, A, B, dY = (t.to(dev) for t in (case.X, case.A, case.B, case.dY))
+    ws = q.new_workspace(case.M, case.K, case.N, case.r, dev)
+    Wp = q.qlora_quantize_nf4(W)
+    Y = torch.empty(case.M, case.N, dtype=torch.bfloat16, device=dev)
+    T = torch.empty(case.M, case.r, dtype=torch.float32, device=dev)
+    dX = torch.empty(case.M, case.K, dtype=torch.bfloat16, device=dev)
+    dA = torch.empty(case.K, case.r, dtype=torch.float32, device=dev)
+    dB = torch.empty(case.r, case.N, dtype=torch.float32, device=dev)
+
+    def step():
+        q.qlora_quantize_nf4(W, out=Wp)
+        q.qlora_linear_fwd(X, Wp, A, B, case.scale, workspace=ws, Y=Y, T_save=T)
+        q.qlora_linear_bwd(dY, X, T, Wp, A, B, case.scale, workspace=ws, dX=dX, dA=dA, dB=dB)
+
+    for _ in range(5):
+        step()
+    stream = torch.cuda.current_stream()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(iters)]
+    for i in range(iters):
+        flush.zero_()
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    if q.qlora_check_status(ws) != 0:
+        raise RuntimeError("device pipeline timeout (tiny)")
+    us = sorted(a.elapsed_time(b) * 1e3 for a, b in evs)[iters // 2]
+    fl = flops_fwd(case.M, case.K, case.N, case.r) + flops_bwd(case.M, case.K, case.N, case.r)
+    return {"workload": "single_qlora_linear_256x256", "M": case.M, "K": case.K, "N": case.N, "r": case.r,
+            "step": "quantize_nf4 + linear_fwd + linear_bwd", "us_per_step": us, "launches_per_step": 3,
+            "gflops": fl / (us * 1e-6) / 1e9, "note": "launch-bound (median of 50 steps, L2 flushed)"}
+
+
 # ---------------------------------------------------------------- small-M sweep
 def small_m_sweep(q, synthetic, dev, flush, iters=10):
     """Small-M forward (W [N x 8192] NF4, M tokens, r = 64): NF4 weight bytes
@@ -771,6 +812,7 @@ def run_ours(args, rank, world, local_rank):
     trio = bench_trio(args, q, synthetic, dev, flush, peaks, local_rank) if extra and not args.block_only else None
     attn = bench_attn(args, q, synthetic, dev, flush, peaks, local_rank) if extra and not args.block_only else None
     small_m = small_m_sweep(q, synthetic, dev, flush) if (extra and not args.no_small_m) else None
+    tiny = bench_tiny(args, q, synthetic, dev, flush) if extra and not args.block_only else None
     if rank != 0:
         return
     cpu = cpu_oracle_block_sample(rows=256, slab=256) if (world == 1 and not args.no_cpu_baseline) else None
@@ -786,7 +828,7 @@ def run_ours(args, rank, world, local_rank):
         "clocks": blk["clocks"], "cpu_baseline": cpu,
         "grad_allreduce_bytes_per_step": blk["grad_bucket_bytes"] if world > 1 else 0,
         "paged_adamw": blk["paged_adamw"],
-        "mlp_trio": trio, "attn_proj": attn, "small_m": small_m,
+        "mlp_trio": trio, "attn_proj": attn, "small_m": small_m, "tiny": tiny,
     }
     print(json.dumps(line), flush=True)
 

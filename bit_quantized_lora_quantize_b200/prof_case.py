@@ -3,6 +3,8 @@
     python -m bit_quantized_lora_quantize_b200.prof_case quantize --n 22016 --k 8192
     python -m bit_quantized_lora_quantize_b200.prof_case fwd --m 16 --n 8192 --k 8192
     python -m bit_quantized_lora_quantize_b200.prof_case bwd --m 4096 --n 4096 --k 4096
+    python -m bit_quantized_lora_quantize_b200.prof_case adamw --n 9994240
+    python -m bit_quantized_lora_quantize_b200.prof_case silu --m 8192 --n 11008
 
 Each case makes its inputs once, runs `--warmup` calls, then `--iters` calls
 with a 256 MB buffer written between them (so the weight is read from HBM, not
@@ -21,7 +23,7 @@ from . import synthetic
 
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
-    ap.add_argument("op", choices=["quantize", "dequantize", "fwd", "bwd"])
+    ap.add_argument("op", choices=["quantize", "dequantize", "fwd", "bwd", "adamw", "silu"])
     ap.add_argument("--m", type=int, default=4096, help="tokens")
     ap.add_argument("--n", type=int, default=4096, help="weight rows (out features)")
     ap.add_argument("--k", type=int, default=4096, help="weight columns (in features)")
@@ -35,7 +37,18 @@ def main(argv=None):
     dev = "cuda:0"
     torch.cuda.set_device(0)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    if a.op in ("quantize", "dequantize"):
+    if a.op == "adamw":
+        # a flat parameter vector of n (the block's adapters: 9994240)
+        from . import paged
+        opt = paged.PagedAdamW([(a.n, 0, 1)], dev, lr=2e-4, weight_decay=0.01)
+        g = torch.randn(a.n, device=dev)
+        call = lambda: opt.step(g)  # noqa: E731
+    elif a.op == "silu":
+        G = torch.randn(a.m, a.n, device=dev).to(torch.bfloat16)
+        U = torch.randn(a.m, a.n, device=dev).to(torch.bfloat16)
+        H = torch.empty_like(G)
+        call = lambda: q.qlora_silu_gate_fwd(G, U, H)  # noqa: E731
+    elif a.op in ("quantize", "dequantize"):
         W = synthetic.weight_only(a.n, a.k, seed=a.seed).to(dev)
         Wp = q.qlora_quantize_nf4(W)
         if a.op == "quantize":
