@@ -358,8 +358,10 @@ def time_steps(step, steps, flush, world, local_rank, sample_clocks=True):
     return float(t.item()) / steps, clocks
 
 
-def time_e2e(e2e_step, steps, world):
-    """Device time per step of the end-to-end step (host copies included)."""
+def time_e2e(e2e_step, steps, world, after=None):
+    """Device time per step of the end-to-end step (host copies included).
+    `after` makes the timing stream wait for work the step left on other
+    streams, so that it ends inside the timed region."""
     import torch
     import torch.distributed as dist
     for _ in range(2):
@@ -372,6 +374,8 @@ def time_e2e(e2e_step, steps, world):
     e0.record(stream)
     for _ in range(steps):
         e2e_step()
+    if after is not None:
+        after()
     e1.record(stream)
     torch.cuda.synchronize()
     t = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device="cuda")
@@ -523,19 +527,82 @@ def bench_block(args, q, synthetic, dp, dev, rank, world, local_rank, flush, pea
     h2d = sum(t.numel() * 2 for t in hW + hdY) + hX.numel() * 2 + hXd.numel() * 2
     d2h = sum(t.numel() * 2 for t in hY + hdX) + hG.numel() * 4
 
-    def e2e_step():
-        for l, w, dy in zip(lins, hW, hdY):
-            l.W.copy_(w, non_blocking=True)
-            l.dY.copy_(dy, non_blocking=True)
-        X.copy_(hX, non_blocking=True)
-        Xd.copy_(hXd, non_blocking=True)
-        step()
-        for l, y, dx in zip(lins, hY, hdX):
-            y.copy_(l.Y, non_blocking=True)
-            dx.copy_(l.dX, non_blocking=True)
-        hG.copy_(bucket.flat, non_blocking=True)
+    # Three streams: host->device copies, the library calls, device->host
+    # copies; per-linear events order them, so the two copy directions and
+    # the kernels overlap (within a step and across steps) and every buffer
+    # is reused only after its previous use.
+    comp = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    n = len(lins)
+    w_ready, w_free = [ev() for _ in range(n)], [ev() for _ in range(n)]
+    dy_ready, dy_free = [ev() for _ in range(n)], [ev() for _ in range(n)]
+    y_done, y_free = [ev() for _ in range(n)], [ev() for _ in range(n)]
+    dx_done, dx_free = [ev() for _ in range(n)], [ev() for _ in range(n)]
+    x_ready, x_free, g_done, g_free = ev(), ev(), ev(), ev()
+    state = {"first": True}
 
-    e2e_ms = time_e2e(e2e_step, args.steps, world)
+    def e2e_step():
+        first = state["first"]
+        state["first"] = False
+        with torch.cuda.stream(s_in):
+            if not first:
+                s_in.wait_event(x_free)
+            X.copy_(hX, non_blocking=True)
+            Xd.copy_(hXd, non_blocking=True)
+            x_ready.record(s_in)
+            for i, (l, w) in enumerate(zip(lins, hW)):
+                if not first:
+                    s_in.wait_event(w_free[i])
+                l.W.copy_(w, non_blocking=True)
+                w_ready[i].record(s_in)
+            for i in reversed(range(n)):
+                if not first:
+                    s_in.wait_event(dy_free[i])
+                lins[i].dY.copy_(hdY[i], non_blocking=True)
+                dy_ready[i].record(s_in)
+        for i, l in enumerate(lins):
+            comp.wait_event(w_ready[i])
+            q.qlora_quantize_nf4(l.W, out=l.P)
+            w_free[i].record(comp)
+        comp.wait_event(x_ready)
+        for i, l in enumerate(lins):
+            if not first:
+                comp.wait_event(y_free[i])
+            q.qlora_linear_fwd(l.X, l.P, l.A, l.B, l.s, workspace=l.ws, Y=l.Y, T_save=l.T)
+            y_done[i].record(comp)
+        if not first:
+            comp.wait_event(g_free)
+        for i in reversed(range(n)):
+            l = lins[i]
+            comp.wait_event(dy_ready[i])
+            if not first:
+                comp.wait_event(dx_free[i])
+            q.qlora_linear_bwd(l.dY, l.X, l.T, l.P, l.A, l.B, l.s, workspace=l.ws, dX=l.dX, dA=l.dA, dB=l.dB)
+            dy_free[i].record(comp)
+            dx_done[i].record(comp)
+        x_free.record(comp)
+        if world > 1:
+            bucket.all_reduce()
+        g_done.record(comp)
+        with torch.cuda.stream(s_out):
+            for i, (l, y) in enumerate(zip(lins, hY)):
+                s_out.wait_event(y_done[i])
+                y.copy_(l.Y, non_blocking=True)
+                y_free[i].record(s_out)
+            for i in reversed(range(n)):
+                s_out.wait_event(dx_done[i])
+                hdX[i].copy_(lins[i].dX, non_blocking=True)
+                dx_free[i].record(s_out)
+            s_out.wait_event(g_done)
+            hG.copy_(bucket.flat, non_blocking=True)
+            g_free.record(s_out)
+
+    def e2e_flush():
+        # The last step's copies out end before the timed region closes.
+        comp.wait_stream(s_out)
+
+    e2e_ms = time_e2e(e2e_step, args.steps, world, after=e2e_flush)
     for l in lins:
         if q.qlora_check_status(l.ws) != 0:
             raise RuntimeError("device pipeline timeout during timing")
@@ -550,7 +617,8 @@ def bench_block(args, q, synthetic, dp, dev, rank, world, local_rank, flush, pea
         "gpu_launches": launches_per_step * args.steps,
         "e2e": {"value": fl_step * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
-                "copies": "in: 7 bf16 weights, X, X_down, 7 dY; out: 7 Y, 7 dX, dA|dB bucket"},
+                "copies": "in: 7 bf16 weights, X, X_down, 7 dY; out: 7 Y, 7 dX, dA|dB bucket; "
+                          "copy streams in each direction overlapped with the kernels"},
         "grad_bucket_bytes": bucket.nbytes, "paged_adamw": opt,
     }
     del lins, bucket, hW, hdY, hY, hdX
