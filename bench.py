@@ -482,18 +482,35 @@ def make_block(q, synthetic, dev, rank, grads_bucket_cls):
     return lins, bucket, X, Xd
 
 
-def block_step_fn(q, lins, calls, bucket, world):
+def block_step_fn(q, lins, calls, bucket, world, streams=None):
+    """The block step.  With `streams` (two CUDA streams, the first the
+    current one) the seven linears' forward+backward chains alternate between
+    them: the linears are independent, so one GEMM's last partial wave
+    overlaps the next one's first tiles.  Each linear keeps its own
+    workspace, and its forward and backward stay on one stream."""
+    import torch
+
+    def on(i):
+        return streams[i % 2] if streams else torch.cuda.current_stream()
+
     def step():
         for l in lins:
             calls("quantize_nf4", l.tag, {"bytes": quantize_bytes(l.numel)},
                   lambda l=l: q.qlora_quantize_nf4(l.W, out=l.P))
-        for l in lins:
-            calls("fused_nf4_fwd", l.tag, {"flops": 2 * l.M * l.N * l.K + 2 * l.M * l.r * (l.N + l.K)},
-                  lambda l=l: q.qlora_linear_fwd(l.X, l.P, l.A, l.B, l.s, workspace=l.ws, Y=l.Y, T_save=l.T))
-        for l in reversed(lins):
-            calls("fused_nf4_dx", l.tag, {"flops": 2 * l.M * l.N * l.K + 2 * l.M * l.r * (l.N + l.K)},
-                  lambda l=l: q.qlora_linear_bwd(l.dY, l.X, l.T, l.P, l.A, l.B, l.s, workspace=l.ws, dX=l.dX,
-                                                 dA=l.dA, dB=l.dB))
+        if streams:
+            streams[1].wait_stream(streams[0])
+        for i, l in enumerate(lins):
+            with torch.cuda.stream(on(i)):
+                calls("fused_nf4_fwd", l.tag, {"flops": 2 * l.M * l.N * l.K + 2 * l.M * l.r * (l.N + l.K)},
+                      lambda l=l: q.qlora_linear_fwd(l.X, l.P, l.A, l.B, l.s, workspace=l.ws, Y=l.Y, T_save=l.T))
+        for i in reversed(range(len(lins))):
+            l = lins[i]
+            with torch.cuda.stream(on(i)):
+                calls("fused_nf4_dx", l.tag, {"flops": 2 * l.M * l.N * l.K + 2 * l.M * l.r * (l.N + l.K)},
+                      lambda l=l: q.qlora_linear_bwd(l.dY, l.X, l.T, l.P, l.A, l.B, l.s, workspace=l.ws, dX=l.dX,
+                                                     dA=l.dA, dB=l.dB))
+        if streams:
+            streams[0].wait_stream(streams[1])
         if world > 1:
             bucket.all_reduce()
     return step
@@ -503,7 +520,12 @@ def bench_block(args, q, synthetic, dp, dev, rank, world, local_rank, flush, pea
     import torch
     lins, bucket, X, Xd = make_block(q, synthetic, dev, rank, dp.GradBucket)
     calls = Calls()
-    step = block_step_fn(q, lins, calls, bucket, world)
+    streams = None if args.one_stream else (torch.cuda.current_stream(), torch.cuda.Stream())
+    step = block_step_fn(q, lins, calls, bucket, world, streams)
+    # Per-launch durations (roofline, kernel table) come from the same step
+    # with every launch on one stream: concurrent launches would share the
+    # GPU inside each other's events.
+    step_serial = block_step_fn(q, lins, calls, bucket, world, None)
     fl_step = sum(flops_fwd(l.M, l.K, l.N, l.r) + flops_bwd(l.M, l.K, l.N, l.r) for l in lins)
     for _ in range(max(3, args.warmup)):
         step()
@@ -512,7 +534,7 @@ def bench_block(args, q, synthetic, dp, dev, rank, world, local_rank, flush, pea
         if q.qlora_check_status(l.ws) != 0:
             raise RuntimeError("device pipeline timeout during warm-up")
     ms, clocks = time_steps(step, args.steps, flush, world, local_rank)
-    agg = calls.profile(step, args.steps, flush)
+    agg = calls.profile(step_serial, args.steps, flush)
 
     # End to end through the public API: every step copies the seven bf16
     # weights, both inputs and the seven dY in from pinned host memory, and
@@ -888,7 +910,8 @@ def run_ours(args, rank, world, local_rank):
         "metric": METRIC, "value": blk["value"], "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": max(3, args.warmup), "ms_per_step": blk["ms_per_step"], "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": dict(BLOCK_WORKLOAD, parallelism=f"dp{world}", global_batch_tokens=M_BLOCK * world, l2=L2_NOTE),
+        "config": dict(BLOCK_WORKLOAD, parallelism=f"dp{world}", global_batch_tokens=M_BLOCK * world, l2=L2_NOTE,
+                       streams=1 if args.one_stream else 2),
         "tokens_per_s": blk["tokens_per_s"], "tflops_dense_only": blk["tflops_dense_only"],
         "flops_per_step": blk["flops_per_step"],
         "roofline": blk["roofline"], "roofline_quantize": blk["roofline_quantize"],
@@ -925,6 +948,7 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-small-m", action="store_true")
     ap.add_argument("--block-only", action="store_true", help="only the headline block step")
+    ap.add_argument("--one-stream", action="store_true", help="the block's linears one after another on one stream")
     args = ap.parse_args(argv)
     if "WORLD_SIZE" not in os.environ and args.gpus > 1:
         # One process per GPU: re-launch under torch.distributed.run.
