@@ -487,16 +487,21 @@ def block_step_fn(q, lins, calls, bucket, world, streams=None):
     current one) the seven linears' forward+backward chains alternate between
     them: the linears are independent, so one GEMM's last partial wave
     overlaps the next one's first tiles.  Each linear keeps its own
-    workspace, and its forward and backward stay on one stream."""
+    workspace, and its forward and backward stay on one stream.  (Putting
+    each weight's quantization at the head of its own chain instead of all
+    seven first measured 0.8 % slower.)"""
     import torch
 
     def on(i):
         return streams[i % 2] if streams else torch.cuda.current_stream()
 
+    def quantize(l):
+        calls("quantize_nf4", l.tag, {"bytes": quantize_bytes(l.numel)},
+              lambda l=l: q.qlora_quantize_nf4(l.W, out=l.P))
+
     def step():
         for l in lins:
-            calls("quantize_nf4", l.tag, {"bytes": quantize_bytes(l.numel)},
-                  lambda l=l: q.qlora_quantize_nf4(l.W, out=l.P))
+            quantize(l)
         if streams:
             streams[1].wait_stream(streams[0])
         for i, l in enumerate(lins):
@@ -718,21 +723,39 @@ def bench_trio(args, q, synthetic, dev, flush, peaks, local_rank):
     calls = Calls()
     fl = lambda K, N: 2 * M * N * K + 2 * M * r * (N + K)  # noqa: E731
 
+    comp = torch.cuda.current_stream()
+    aux = None if args.one_stream else torch.cuda.Stream()
+
+    def pair(f_gate, f_up):
+        # gate and up are independent: with a second stream they run side by
+        # side (their partial last waves overlap), joined before the glue.
+        if aux is None:
+            f_gate()
+            f_up()
+            return
+        aux.wait_stream(comp)
+        f_gate()
+        with torch.cuda.stream(aux):
+            f_up()
+        comp.wait_stream(aux)
+
     def step():
-        calls("fused_nf4_fwd", "gate", {"flops": fl(D, Fd)},
-              lambda: q.qlora_linear_fwd(X, Pg, Ag, Bg, s, workspace=wsg, Y=G, T_save=Tg))
-        calls("fused_nf4_fwd", "up", {"flops": fl(D, Fd)},
-              lambda: q.qlora_linear_fwd(X, Pu, Au, Bu, s, workspace=wsu, Y=Up, T_save=Tu))
+        pair(lambda: calls("fused_nf4_fwd", "gate", {"flops": fl(D, Fd)},
+                           lambda: q.qlora_linear_fwd(X, Pg, Ag, Bg, s, workspace=wsg, Y=G, T_save=Tg)),
+             lambda: calls("fused_nf4_fwd", "up", {"flops": fl(D, Fd)},
+                           lambda: q.qlora_linear_fwd(X, Pu, Au, Bu, s, workspace=wsu, Y=Up, T_save=Tu)))
         calls("silu_gate_fwd", "trio", {"bytes": 3 * 2 * M * Fd}, lambda: q.qlora_silu_gate_fwd(G, Up, H))
         calls("fused_nf4_fwd", "down", {"flops": fl(Fd, D)},
               lambda: q.qlora_linear_fwd(H, Pd, Ad, Bd, s, workspace=wsd, Y=Y, T_save=Td))
         calls("fused_nf4_dx", "down", {"flops": fl(Fd, D)},
               lambda: q.qlora_linear_bwd(dY, H, Td, Pd, Ad, Bd, s, workspace=wsd, dX=dH, dA=gA[2], dB=gB[2]))
         calls("silu_gate_bwd", "trio", {"bytes": 5 * 2 * M * Fd}, lambda: q.qlora_silu_gate_bwd(G, Up, dH, dG, dU))
-        calls("fused_nf4_dx", "gate", {"flops": fl(D, Fd)},
-              lambda: q.qlora_linear_bwd(dG, X, Tg, Pg, Ag, Bg, s, workspace=wsg, dX=dXg, dA=gA[0], dB=gB[0]))
-        calls("fused_nf4_dx", "up", {"flops": fl(D, Fd)},
-              lambda: q.qlora_linear_bwd(dU, X, Tu, Pu, Au, Bu, s, workspace=wsu, dX=dXu, dA=gA[1], dB=gB[1]))
+        pair(lambda: calls("fused_nf4_dx", "gate", {"flops": fl(D, Fd)},
+                           lambda: q.qlora_linear_bwd(dG, X, Tg, Pg, Ag, Bg, s, workspace=wsg, dX=dXg, dA=gA[0],
+                                                      dB=gB[0])),
+             lambda: calls("fused_nf4_dx", "up", {"flops": fl(D, Fd)},
+                           lambda: q.qlora_linear_bwd(dU, X, Tu, Pu, Au, Bu, s, workspace=wsu, dX=dXu, dA=gA[1],
+                                                      dB=gB[1])))
         torch.add(dXg, dXu, out=dX)  # the input's two gradient paths (torch add, bf16)
 
     fl_step = 2 * (flops_fwd(M, D, Fd, r) + flops_bwd(M, D, Fd, r)) + flops_fwd(M, Fd, D, r) + flops_bwd(M, Fd, D, r)
@@ -740,7 +763,9 @@ def bench_trio(args, q, synthetic, dev, flush, peaks, local_rank):
         step()
     torch.cuda.synchronize()
     ms, clocks = time_steps(step, args.steps, flush, 1, local_rank)
+    aux_saved, aux = aux, None  # per-launch events on one stream
     agg = calls.profile(step, args.steps, flush)
+    aux = aux_saved
     hX, hdY = t.X.pin_memory(), t.dY.pin_memory()
     hY = torch.empty(Y.shape, dtype=bf).pin_memory()
     hdX = torch.empty(M, D, dtype=bf).pin_memory()
