@@ -17,7 +17,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(PKG, "csrc")
 ROOT = os.path.dirname(PKG)
 LIB = os.path.join(PKG, "libqlora.so")
-SOURCES = ["abi.cu", "fused_pair.cu", "smallm.cu", "quantize.cu", "nf4_host.cu", "noalloc.cu", "glue.cu", "adamw.cu"]
+SOURCES = ["abi.cu", "fused_pair.cu", "smallm.cu", "smallm_rd.cu", "quantize.cu", "nf4_host.cu", "noalloc.cu", "glue.cu", "adamw.cu"]
 HEADERS = ["ptx.cuh", "nf4_device.cuh", "kernels.h", "tensor_map.h", "nf4_host.h", "abi_internal.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden"]

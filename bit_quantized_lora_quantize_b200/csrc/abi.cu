@@ -40,10 +40,14 @@ int rank8(int r) { return (r + 7) / 8 * 8; }
 // The weight-streaming forward holds rank indices in one 128-row MMA tile.
 bool small_m_path(int64_t M, int r) { return M <= kSmallMMax && rank8(r) <= 128; }
 
+// Up to 16 tokens the forward decodes into register fragments of mma.sync
+// (smallm_rd.cu); beyond that, up to 128, into tensor memory (smallm.cu).
+bool small_m_rd_path(int64_t M, int r) { return M <= kSmallMRdMax && rank8(r) <= 128; }
+
 // Workspace: [status word (256 B)][counters of the forward and input-gradient
-// GEMMs][T pair: bf16 M x 2rp][U pair: bf16 M x 2rp]; when the small-M
-// forward runs, [its counters and partial tiles]; when r % 8 != 0, [A, B, T,
-// dA, dB padded to r8].
+// GEMMs][T pair: bf16 M x 2rp][U pair: bf16 M x 2rp]; when a small-M
+// forward runs, [its counters, partials and float32 partial of Y]; when
+// r % 8 != 0, [A, B, T, dA, dB padded to r8].
 struct WsLayout {
   size_t cf_off, cd_off, t_off, u_off, sm_off, pad_off;
   size_t pa_off, pb_off, pt_off, pda_off, pdb_off, total;
@@ -59,7 +63,12 @@ WsLayout ws_layout(int64_t M, int64_t K, int64_t N, int r) {
   w.t_off = w.cd_off + ctr_bytes;
   w.u_off = w.t_off + pair_bytes;
   w.sm_off = w.u_off + pair_bytes;
-  w.pad_off = w.sm_off + (small_m_path(M, r) ? round_up(small_m_workspace_bytes(M, N, r8), 256) : 0);
+  size_t sm_bytes = 0;
+  if (small_m_rd_path(M, r))
+    sm_bytes = small_m_rd_workspace_bytes(M, K, N, r8);
+  else if (small_m_path(M, r))
+    sm_bytes = small_m_workspace_bytes(M, N, r8);
+  w.pad_off = w.sm_off + round_up(sm_bytes, 256);
   size_t o = w.pad_off;
   if (r8 != r) {
     w.pa_off = o; o += round_up(static_cast<size_t>(K) * r8 * 2, 256);
@@ -170,6 +179,23 @@ bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, 
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool make_map_nd(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, int rank, const uint64_t* dims,
+                 const uint64_t* strides_bytes, const uint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || rank < 1 || rank > 5) return false;
+  cuuint64_t d[5], st[4];
+  cuuint32_t b[5], e[5];
+  for (int i = 0; i < rank; ++i) {
+    d[i] = static_cast<cuuint64_t>(dims[i]);
+    b[i] = static_cast<cuuint32_t>(box[i]);
+    e[i] = 1;
+  }
+  for (int i = 0; i + 1 < rank; ++i) st[i] = static_cast<cuuint64_t>(strides_bytes[i]);
+  return fn(map, dtype, static_cast<cuuint32_t>(rank), const_cast<void*>(base), d, st, b, e,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace qlora
 
 using namespace qlora;
@@ -264,7 +290,13 @@ qlora_status qlora_linear_fwd_4bit(const uint16_t* X, int64_t M, int64_t K, int6
     Tk = reinterpret_cast<float*>(ws + wl.pt_off);
   }
   cudaError_t e;
-  if (small_m_path(M, r)) {
+  if (small_m_rd_path(M, r)) {
+    // Three launches: T, the weight stream, Y = bf16(stream + T B).
+    ProfScope p0(st, "small_m_nf4_fwd", 3);
+    e = launch_small_m_rd(X, codes, absmax_q, absmax_scale, Ak, Bk, M, K, N, r8, scale, Y, Tk, ws + wl.sm_off, status,
+                          P, st);
+    p0.done();
+  } else if (small_m_path(M, r)) {
     // One launch: T, its pair and Y.
     ProfScope p0(st, "small_m_nf4_fwd", 1);
     e = launch_small_m_fwd(X, codes, absmax_q, absmax_scale, Ak, Bk, M, K, N, r8, scale, Y, Tk, Tpair,

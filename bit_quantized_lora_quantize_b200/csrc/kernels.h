@@ -82,6 +82,18 @@ cudaError_t launch_small_m_fwd(const uint16_t* X, const uint8_t* codes, const ui
                                int64_t K, int64_t N, int r, float scale, uint16_t* Y, float* T_save, uint16_t* Tpair,
                                void* scratch, int* status, const Nf4Params& P, cudaStream_t stream);
 
+// Small-M forward for M <= kSmallMRdMax tokens and ranks <= 128: T = s X A,
+// the weight stream (float32 partials of Y in `scratch`) and
+// Y = bf16(sum of partials + T B), three launches chained by programmatic
+// dependent launch.  `scratch` holds small_m_rd_workspace_bytes(M, K, N, r)
+// bytes, zero before the first call; the kernels leave their counters at zero.
+constexpr int64_t kSmallMRdMax = 16;
+size_t small_m_rd_workspace_bytes(int64_t M, int64_t K, int64_t N, int r);
+cudaError_t launch_small_m_rd(const uint16_t* X, const uint8_t* codes, const uint8_t* absmax_q,
+                              const float* absmax_scale, const uint16_t* A, const uint16_t* B, int64_t M, int64_t K,
+                              int64_t N, int r, float scale, uint16_t* Y, float* T_save, void* scratch, int* status,
+                              const Nf4Params& P, cudaStream_t stream);
+
 // Copy a rows x src_cols matrix (row stride src_ld elements of elem_bytes,
 // 2 or 4) into dst (row stride dst_ld), filling columns [src_cols, dst_cols)
 // and rows [rows, dst_rows) with zeros (dst_rows = rows when omitted).  Used to

@@ -1,0 +1,644 @@
+// Small-M forward of the NF4 LoRA linear layer for M <= 16 tokens, sm_100a.
+//
+// "QLoRA: Fine-Tuning 65-Billion Parameter Models on a Single Consumer GPU",
+// "QLoRA's Working Process" and its closing remark that 4-bit inference is
+// still slow: with a handful of tokens the forward is a stream over the packed
+// weight.  What bounds such a stream here is the number of bytes in flight
+// per SM and the shared-memory traffic of the decode, so this path:
+//
+//  * streams the codes with TMA in tiles of 256 weight rows x 128 bytes (256
+//    inputs, four 64-input blocks) through a 4-stage ring, 128 KB in flight
+//    per SM, and brings the matching slice of X with one 5-D TMA whose box
+//    lands it in the order the MMA fragments are read in (no multicast);
+//  * decodes a code byte with one byte permute, which forms the address of a
+//    bf16 level pair in a table with 32 bank-private copies, and one 32-bit
+//    shared load;
+//  * multiplies with mma.sync m16n8k16 (bf16 in, float32 accumulate): weight
+//    rows on the 16-row side, tokens on the 8-column side;
+//  * multiplies each 64-input block's partial product by the block constant
+//    (float32) instead of scaling every weight;
+//  * spreads the (256-row block, 256-input chunk) units evenly over one CTA
+//    per SM; each warp stores a float32 partial of every row block it
+//    worked on, with no synchronisation, and the epilogue kernel sums a row
+//    block's partials in a fixed order.
+//
+// T = s X A is computed by the same stream: the rows of A^T are appended to
+// the weight as extra row blocks (bf16, no block constant), so that their
+// products with the X tiles already on chip are partials of T.  A small kernel
+// launched after the stream (programmatic dependent launch) sums the partials
+// into T and Y = bf16(sum of partials + T B).
+//
+// Rounding.  A block's product is sum_k bf16(q_k) x_k (exact products,
+// float32 sums) times the float32 constant a'_b; the other paths multiply by
+// the dequantized weight bf16(fp32(q_k) a'_b).  Each form carries one bf16
+// rounding of relative size <= 2^-9 per term against the exact q_k a'_b x_k.
+#include <algorithm>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "kernels.h"
+#include "nf4_device.cuh"
+#include "ptx.cuh"
+#include "tensor_map.h"
+
+namespace qlora {
+namespace {
+
+constexpr int kRows = 256;                  // weight rows per unit
+constexpr int kKc = 256;                    // inputs per unit (4 blocks, 128 B of codes per row)
+constexpr int kStages = 4;
+constexpr int kCons = 16;                   // consumer warps: row group w & 7, block pair w >> 3
+constexpr int kThreads = (kCons + 1) * 32;  // + one producer warp
+constexpr int kCodeStage = kRows * kKc / 2;
+constexpr int kMaxGridRd = 160;
+
+template <int NT>
+struct RdLayout {
+  static constexpr int MP = 8 * NT;                        // tokens, padded
+  static constexpr int kXStage = MP * kKc * 2;
+  static constexpr int offCodes = 65536;                   // after the 64 KB level-pair table
+  static constexpr int offX = offCodes + kStages * kCodeStage;
+  static constexpr int offLvl = offX + kStages * kXStage;  // 256 float32 constant levels
+  static constexpr int offBar = offLvl + 1024;
+  static constexpr int offAbort = offBar + 2 * kStages * 8;
+  static constexpr int kDynamic = offAbort + 16;
+};
+static_assert(RdLayout<2>::kDynamic <= 232448, "shared memory budget");
+
+struct RdArgs {
+  int M, N, K, KB, CH, RB, RBW, S2;
+  int64_t U;             // units = RB * CH; row blocks RBW.. hold the rows of A^T (T = X A)
+  int64_t n_scales;      // group scales in absmax_scale (the centred mean follows them)
+  const uint8_t* absmax_q;
+  const float* absmax_scale;
+  float* partial;        // [RB][S2][256][MP] float32: one slot per (contributing CTA, block pair)
+  int* status;
+  uint64_t wait_ns;
+  Nf4Params nf4;
+};
+
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+  return v;
+}
+// D = A B (+ 0) and D += A B, m16n8k16, bf16 inputs, float32 accumulators.
+__device__ __forceinline__ void mma_first(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%10,%10,%10,%10};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.0f));
+}
+__device__ __forceinline__ void mma_acc(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Schedule (identical on host and device): CTA j owns units
+// [U j / G, U (j + 1) / G); unit u is (row block u / CH, chunk u % CH).
+__host__ __device__ __forceinline__ int64_t unit_start(int j, int64_t U, int G) { return U * j / G; }
+__host__ __device__ __forceinline__ int cta_of(int64_t u, int64_t U, int G) {
+  return static_cast<int>(((u + 1) * G + U - 1) / U - 1);
+}
+
+// ---------------------------------------------------------------- weight stream
+template <int NT>
+__global__ void __launch_bounds__(kThreads, 1)
+    smallm_rd_kernel(const __grid_constant__ CUtensorMap mapC, const __grid_constant__ CUtensorMap mapX,
+                     const __grid_constant__ CUtensorMap mapA, const RdArgs a) {
+  using L = RdLayout<NT>;
+  constexpr int MP = L::MP;
+  // The kernel has no static shared memory: the dynamic window starts at
+  // shared address 0, aligned for the 128-byte-swizzled TMA tiles.
+  extern __shared__ __align__(1024) uint8_t sm[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + L::offBar);
+  uint64_t* empty = full + kStages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::offAbort);
+  float* lvl2 = reinterpret_cast<float*>(sm + L::offLvl);
+  if (smem_u32(sm) & 1023u) {  // the swizzled copies need a 1024-byte aligned window
+    if (tid == 0 && a.status) atomicCAS(a.status, 0, 0x100 + 62);
+    return;
+  }
+
+  // Level-pair table: entry e (a code byte; the high nibble is the earlier
+  // input) holds bf16(q[e >> 4]) in its low half and bf16(q[e & 15]) in its
+  // high half; entry e, copy l sits at byte e * 256 + 4 l, so lane l always
+  // reads bank l.  The upper 128 bytes of each 256-byte row stay unused.
+  for (int i = tid; i < 256 * 32; i += kThreads) {
+    const int e = i >> 5, l = i & 31;
+    reinterpret_cast<uint32_t*>(sm)[e * 64 + l] = pack_bf16x2_rn(a.nf4.q[e >> 4], a.nf4.q[e & 15]);
+  }
+  for (int i = tid; i < 256; i += kThreads) lvl2[i] = level2_value_for(static_cast<uint32_t>(i), a.nf4.centred);
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kCons);
+    }
+    *abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  __syncthreads();
+  griddep_launch_dependents();  // the epilogue kernel may get resident now; it waits for this grid
+
+  const int G = gridDim.x, j = blockIdx.x;
+  const int64_t u0 = unit_start(j, a.U, G), u1 = unit_start(j + 1, a.U, G);
+  const int nu = static_cast<int>(u1 - u0);
+  const int CH = a.CH;
+
+  if (warp == kCons) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const WaitCtx ctx{abort_flag, a.status, 60, a.wait_ns};
+      tma_prefetch_desc(&mapC);
+      tma_prefetch_desc(&mapX);
+      tma_prefetch_desc(&mapA);
+      int rb = static_cast<int>(u0 / CH), ch = static_cast<int>(u0 % CH);
+      int issued = 0;
+      for (int i = 0; i < nu; ++i) {
+        const int s = i % kStages;
+        if (i >= kStages && !mbar_wait(&empty[s], ((i / kStages) & 1) ^ 1, ctx)) break;
+        mbar_arrive_expect_tx(&full[s], kCodeStage + L::kXStage);
+        if (rb < a.RBW)
+          tma_load_2d(&mapC, &full[s], sm + L::offCodes + s * kCodeStage, ch * 128, rb * kRows);
+        else  // 64 columns of A x 256 inputs, bf16: the same 32 KB
+          tma_load_2d(&mapA, &full[s], sm + L::offCodes + s * kCodeStage, 64 * (rb - a.RBW), ch * kKc);
+        tma_load_5d_outer(&mapX, &full[s], sm + L::offX + s * L::kXStage, 4 * ch);
+        ++issued;
+        if (++ch == CH) {
+          ch = 0;
+          ++rb;
+        }
+      }
+      // After an abort nobody consumes the copies still in flight: they land
+      // before the CTA exits.
+      if (*abort_flag)
+        for (int i = issued > kStages ? issued - kStages : 0; i < issued; ++i)
+          mbar_drain(&full[i % kStages], (i / kStages) & 1);
+    }
+  } else {
+    // ------------------------------------------------------------ consumers
+    const WaitCtx ctx{abort_flag, a.status, 61, a.wait_ns};
+    const int rg = warp & 7, kh = warp >> 3;
+    const int g = lane >> 2, c = lane & 3;
+    const uint32_t lane4 = static_cast<uint32_t>(lane) * 4u;
+    const uint32_t tab = smem_u32(sm);
+    const uint32_t codes0 = smem_u32(sm + L::offCodes), x0 = smem_u32(sm + L::offX);
+    const int KB = a.KB;
+    const float mu = centred_mu(a.absmax_scale, a.n_scales, a.nf4.centred);
+    // This lane loads the constants of row r_own (t = c >> 1, h = c & 1) and
+    // hands them to the lanes that need them.
+    const int r_own = 32 * rg + 16 * (c >> 1) + 8 * (c & 1) + g;
+    const bool vec16 = (KB & 15) == 0 && (reinterpret_cast<uintptr_t>(a.absmax_q) & 15u) == 0;
+    // Raw 8-bit constants and the two group scales of 16 consecutive blocks.
+    auto fetch = [&](int rbx, int gx, uint4& q, float (&sc)[2]) {
+      q = make_uint4(0, 0, 0, 0);
+      sc[0] = sc[1] = 0.0f;
+      const int n = rbx * kRows + r_own;
+      if (rbx >= a.RBW || n >= a.N) return;
+      const int64_t b0 = static_cast<int64_t>(n) * KB + 16 * gx;
+      if (vec16) {
+        q = __ldg(reinterpret_cast<const uint4*>(a.absmax_q + b0));
+      } else {
+        uint32_t w4[4] = {0, 0, 0, 0};
+        for (int e = 0; e < 16 && 16 * gx + e < KB; ++e)
+          w4[e >> 2] |= static_cast<uint32_t>(__ldg(a.absmax_q + b0 + e)) << (8 * (e & 3));
+        q = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+      }
+      const int64_t i0 = b0 >> 8;
+      sc[0] = __ldg(a.absmax_scale + i0);
+      sc[1] = __ldg(a.absmax_scale + (i0 + 1 < a.n_scales ? i0 + 1 : i0));
+    };
+    auto next_group = [&](int rbx, int gx, int& nrb, int& ng) {
+      nrb = rbx;
+      ng = gx + 1;
+      if (ng * 4 >= CH) {
+        ng = 0;
+        ++nrb;
+      }
+    };
+    int rb = static_cast<int>(u0 / CH), ch = static_cast<int>(u0 % CH);
+    uint4 gq, gq_n;
+    float gs[2], gs_n[2];
+    fetch(rb, ch >> 2, gq, gs);
+    {
+      int nrb, ng;
+      next_group(rb, ch >> 2, nrb, ng);
+      fetch(nrb, ng, gq_n, gs_n);
+    }
+    float acc[2][NT][4];
+#pragma unroll
+    for (int t = 0; t < 2; ++t)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[t][nt][e] = 0.0f;
+
+    for (int i = 0; i < nu; ++i) {
+      const int s = i % kStages;
+      // Constants of this unit's two blocks for row r_own.
+      float aown[2];
+      {
+        const int sb = (ch & 3) * 4 + 2 * kh;
+        const uint32_t word = sb < 4 ? gq.x : sb < 8 ? gq.y : sb < 12 ? gq.z : gq.w;
+        const int n = rb * kRows + r_own;
+        const int64_t bl0 = static_cast<int64_t>(n < a.N ? n : 0) * KB + 16 * (ch >> 2);
+#pragma unroll
+        for (int bb = 0; bb < 2; ++bb) {
+          const uint32_t q = (word >> (8 * ((sb + bb) & 3))) & 255u;
+          const float sc = ((bl0 + sb + bb) >> 8) == (bl0 >> 8) ? gs[0] : gs[1];
+          const bool live = n < a.N && ch * 4 + 2 * kh + bb < KB;
+          aown[bb] = live ? __fadd_rn(__fmul_rn(lvl2[q], sc), mu) : 0.0f;
+        }
+      }
+      int nrb = rb, nch = ch + 1;
+      if (nch == CH) {
+        nch = 0;
+        ++nrb;
+      }
+      if ((nch & 3) == 0) {  // the next unit starts the next group: rotate, fetch the one after
+        gq = gq_n;
+        gs[0] = gs_n[0];
+        gs[1] = gs_n[1];
+        int rr, ng;
+        next_group(nrb, nch >> 2, rr, ng);
+        fetch(rr, ng, gq_n, gs_n);
+      }
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&full[s], (i / kStages) & 1, ctx))) break;
+
+      const uint32_t cs = codes0 + s * kCodeStage, xs = x0 + s * L::kXStage;
+      if (rb >= a.RBW) {
+        // Rows of A^T: the stage holds A[256 inputs][64 columns] bf16 with the
+        // 128-byte swizzle; row j of A^T, inputs k..k+3 are 4 scalars of it.
+        // No block constant.  Row groups 0 and 1 cover the 64 columns.
+        if (rg < 2) {
+#pragma unroll
+          for (int s4 = 0; s4 < 4; ++s4) {
+#pragma unroll
+            for (int bb = 0; bb < 2; ++bb) {
+              const int b = 2 * kh + bb;
+              const int k0 = 64 * b + 16 * c + 4 * s4;
+              uint32_t A[2][4];
+#pragma unroll
+              for (int t = 0; t < 2; ++t)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                  const int jj = 32 * rg + 16 * t + 8 * h + g;
+                  uint32_t v[4];
+#pragma unroll
+                  for (int e = 0; e < 4; ++e) {
+                    const int k = k0 + e;
+                    uint16_t x;
+                    asm volatile("ld.shared.u16 %0, [%1];"
+                                 : "=h"(x)
+                                 : "r"(cs + k * 128 + ((((jj >> 3) ^ (k & 7)) & 7) << 4) + (jj & 7) * 2));
+                    v[e] = x;
+                  }
+                  A[t][h] = v[0] | (v[1] << 16);
+                  A[t][h + 2] = v[2] | (v[3] << 16);
+                }
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt) {
+                const uint2 xb = lds64(xs + (((b * 2 + (s4 >> 1)) * MP + 8 * nt + g) * 4 + c) * 16 + 8 * (s4 & 1));
+                mma_acc(acc[0][nt], A[0], xb.x, xb.y);
+                mma_acc(acc[1][nt], A[1], xb.x, xb.y);
+              }
+            }
+          }
+        }
+      } else {
+      float av[2][2][2];  // [t][h][bb]
+#pragma unroll
+      for (int bb = 0; bb < 2; ++bb)
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+          for (int h = 0; h < 2; ++h) av[t][h][bb] = __shfl_sync(0xFFFFFFFFu, aown[bb], g * 4 + t * 2 + h);
+      // This lane's 8 code bytes per (block, row): inputs 16c .. 16c + 15 of
+      // the block; the 128-byte swizzle puts 16-byte chunk k of row r at k ^ (r & 7).
+      uint2 w[2][2][2];  // [bb][t][h]
+#pragma unroll
+      for (int bb = 0; bb < 2; ++bb)
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int r = 32 * rg + 16 * t + 8 * h + g, b = 2 * kh + bb;
+            w[bb][t][h] = lds64(cs + r * 128 + (((2 * b + (c >> 1)) ^ g) << 4) + 8 * (c & 1));
+          }
+      float bl[2][2][NT][4];  // [bb][t][nt]
+#pragma unroll
+      for (int s4 = 0; s4 < 4; ++s4) {
+#pragma unroll
+        for (int bb = 0; bb < 2; ++bb) {
+          const int b = 2 * kh + bb;
+          // MMA k-slots 2c, 2c+1 <- inputs 16c + 4 s4 + {0, 1} (code byte 2 s4),
+          // slots 2c+8, 2c+9 <- inputs 16c + 4 s4 + {2, 3} (code byte 2 s4 + 1).
+          const uint32_t j0 = (2 * s4) & 3;
+          uint32_t A[2][4];
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            const uint32_t w0 = s4 < 2 ? w[bb][t][0].x : w[bb][t][0].y;
+            const uint32_t w1 = s4 < 2 ? w[bb][t][1].x : w[bb][t][1].y;
+            A[t][0] = lds32(tab + prmt(w0, lane4, 0x5504u | (j0 << 4)));
+            A[t][1] = lds32(tab + prmt(w1, lane4, 0x5504u | (j0 << 4)));
+            A[t][2] = lds32(tab + prmt(w0, lane4, 0x5504u | ((j0 + 1) << 4)));
+            A[t][3] = lds32(tab + prmt(w1, lane4, 0x5504u | ((j0 + 1) << 4)));
+          }
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            // X tile layout [block][s4 / 2][token][c][8 inputs].
+            const uint2 xb = lds64(xs + (((b * 2 + (s4 >> 1)) * MP + 8 * nt + g) * 4 + c) * 16 + 8 * (s4 & 1));
+            if (s4 == 0) {
+              mma_first(bl[bb][0][nt], A[0], xb.x, xb.y);
+              mma_first(bl[bb][1][nt], A[1], xb.x, xb.y);
+            } else {
+              mma_acc(bl[bb][0][nt], A[0], xb.x, xb.y);
+              mma_acc(bl[bb][1][nt], A[1], xb.x, xb.y);
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int bb = 0; bb < 2; ++bb)
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            acc[t][nt][0] = fmaf(av[t][0][bb], bl[bb][t][nt][0], acc[t][nt][0]);
+            acc[t][nt][1] = fmaf(av[t][0][bb], bl[bb][t][nt][1], acc[t][nt][1]);
+            acc[t][nt][2] = fmaf(av[t][1][bb], bl[bb][t][nt][2], acc[t][nt][2]);
+            acc[t][nt][3] = fmaf(av[t][1][bb], bl[bb][t][nt][3], acc[t][nt][3]);
+          }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+
+      if (nrb != rb || i + 1 == nu) {
+        // Row block rb ends here for this warp: store its part of row group
+        // rg in the slot of (this CTA, block pair); the epilogue kernel sums
+        // the slots of each row block in order.
+        const int jf = cta_of(static_cast<int64_t>(rb) * CH, a.U, G);
+        if (rb < a.RBW || rg < 2) {
+        float* my = a.partial + ((static_cast<int64_t>(rb) * a.S2 + 2 * (j - jf) + kh) * kRows + 32 * rg) * MP;
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            *reinterpret_cast<float2*>(my + (16 * t + g) * MP + 8 * nt + 2 * c) =
+                make_float2(acc[t][nt][0], acc[t][nt][1]);
+            *reinterpret_cast<float2*>(my + (16 * t + g + 8) * MP + 8 * nt + 2 * c) =
+                make_float2(acc[t][nt][2], acc[t][nt][3]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[t][nt][e] = 0.0f;
+          }
+        }
+      }
+      rb = nrb;
+      ch = nch;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- Y = bf16(partials + T B)
+// Warp: 8 adjacent outputs n (four pairs) of four tokens.  Lane (pair p,
+// slice q) sums the partial slots q, q + 8, ... of the output's row block and
+// ranks q r/8 .. (q + 1) r/8 - 1 of T B, then a fixed butterfly over the 8
+// slices completes the sum.
+struct UpArgs {
+  int M, N, r, CH, G, S2, MP, RBW;
+  int64_t U;
+  float scale;
+};
+
+// Sum, in slot order, the partials of row `row` of row block rb for token m.
+__device__ __forceinline__ float sum_partials(const float* partial, const UpArgs& u, int rb, int row, int m) {
+  const int jf = cta_of(static_cast<int64_t>(rb) * u.CH, u.U, u.G);
+  const int jl = cta_of(static_cast<int64_t>(rb + 1) * u.CH - 1, u.U, u.G);
+  float v = 0.0f;
+  for (int p = 0; p < 2 * (jl - jf + 1); ++p)
+    v += __ldcg(partial + ((static_cast<int64_t>(rb) * u.S2 + p) * kRows + row) * u.MP + m);
+  return v;
+}
+
+__global__ void __launch_bounds__(256) lora_up_kernel(float* __restrict__ T, const uint16_t* __restrict__ B,
+                                                      const float* __restrict__ partial, const UpArgs u,
+                                                      uint16_t* __restrict__ Y) {
+  const int lane = threadIdx.x & 31, q = lane & 7, p = lane >> 3;
+  const int n = (blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5)) * 8 + 2 * p;
+  const int m0 = blockIdx.y * 4;
+  const bool live = n < u.N;
+  const int rs = u.r / 8;  // r is a multiple of 8, at most 128
+  // B is an input of the call: read it before waiting for the stream.
+  uint32_t bw[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e)
+    bw[e] = live && e < rs ? __ldg(reinterpret_cast<const uint32_t*>(B + static_cast<int64_t>(q * rs + e) * u.N + n)) : 0u;
+  griddep_wait();  // the weight stream has completed
+  // This CTA's four rows of T = s X A, summed from the A^T row blocks'
+  // partials (the CTAs of the first column also store T for the backward);
+  // the partial slots of Y are read in the same round.
+  __shared__ float Ts[4][128];
+  for (int i = threadIdx.x; i < 4 * u.r; i += blockDim.x) {
+    const int mm = i / u.r, jj = i % u.r;
+    float t = 0.0f;
+    if (m0 + mm < u.M) {
+      t = __fmul_rn(u.scale, sum_partials(partial, u, u.RBW + jj / 64, jj % 64, m0 + mm));
+      if (blockIdx.x == 0) T[static_cast<int64_t>(m0 + mm) * u.r + jj] = t;
+    }
+    Ts[mm][jj] = t;
+  }
+  float z[4][2];
+#pragma unroll
+  for (int mm = 0; mm < 4; ++mm) z[mm][0] = z[mm][1] = 0.0f;
+  if (live) {
+    const int rb = n / kRows, row = n % kRows;
+    const int jf = cta_of(static_cast<int64_t>(rb) * u.CH, u.U, u.G);
+    const int jl = cta_of(static_cast<int64_t>(rb + 1) * u.CH - 1, u.U, u.G);
+    const int nparts = 2 * (jl - jf + 1);
+    for (int s = q; s < nparts; s += 8) {
+      const float* ps = partial + ((static_cast<int64_t>(rb) * u.S2 + s) * kRows + row) * u.MP + m0;
+      const float4 v0 = __ldcg(reinterpret_cast<const float4*>(ps));
+      const float4 v1 = __ldcg(reinterpret_cast<const float4*>(ps + u.MP));
+      z[0][0] += v0.x; z[1][0] += v0.y; z[2][0] += v0.z; z[3][0] += v0.w;
+      z[0][1] += v1.x; z[1][1] += v1.y; z[2][1] += v1.z; z[3][1] += v1.w;
+    }
+  }
+  __syncthreads();
+  if (live) {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      if (e < rs) {
+        const float b0 = __uint_as_float(bw[e] << 16), b1 = __uint_as_float(bw[e] & 0xFFFF0000u);
+#pragma unroll
+        for (int mm = 0; mm < 4; ++mm) {
+          const float t = Ts[mm][q * rs + e];
+          z[mm][0] = fmaf(t, b0, z[mm][0]);
+          z[mm][1] = fmaf(t, b1, z[mm][1]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 1; o < 8; o <<= 1)
+#pragma unroll
+    for (int mm = 0; mm < 4; ++mm) {
+      z[mm][0] += __shfl_xor_sync(0xFFFFFFFFu, z[mm][0], o);
+      z[mm][1] += __shfl_xor_sync(0xFFFFFFFFu, z[mm][1], o);
+    }
+  if (!live || q != 0) return;
+#pragma unroll
+  for (int mm = 0; mm < 4; ++mm) {
+    const int m = m0 + mm;
+    if (m < u.M) *reinterpret_cast<uint32_t*>(Y + static_cast<int64_t>(m) * u.N + n) = pack_bf16x2_rn(z[mm][0], z[mm][1]);
+  }
+}
+
+int rd_sm_count() {
+  static int cached[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!cached[dev]) {
+    int v = 0;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    cached[dev] = v > 0 ? v : 148;
+  }
+  return cached[dev];
+}
+
+struct RdPlan {
+  int KB, CH, RB, RBW, G, S2, MP;
+  int64_t U;
+  size_t off_partial, total;
+};
+
+size_t r256(size_t x) { return (x + 255) / 256 * 256; }
+
+RdPlan rd_plan(int64_t M, int64_t K, int64_t N, int r, int sms) {
+  RdPlan p{};
+  p.KB = static_cast<int>(K / 64);
+  p.CH = static_cast<int>((K + kKc - 1) / kKc);
+  p.RBW = static_cast<int>((N + kRows - 1) / kRows);
+  p.RB = p.RBW + (r + 63) / 64;  // + the rows of A^T, 64 per block
+  p.U = static_cast<int64_t>(p.RB) * p.CH;
+  p.G = static_cast<int>(std::min<int64_t>({static_cast<int64_t>(sms), static_cast<int64_t>(kMaxGridRd), p.U}));
+  // A row block spans at most ceil(CH / (U / G)) + 1 CTAs.
+  const int64_t per = p.U / p.G;  // >= 1
+  const int maxc = static_cast<int>(std::min<int64_t>(p.G, (p.CH + per - 1) / per + 1));
+  p.S2 = 2 * maxc;
+  p.MP = M <= 8 ? 8 : 16;
+  size_t o = 0;
+  p.off_partial = o;
+  o += r256(static_cast<size_t>(p.RB) * p.S2 * kRows * p.MP * 4);
+  p.total = o;
+  return p;
+}
+
+template <int NT>
+cudaError_t launch_rd_main(const CUtensorMap& mC, const CUtensorMap& mX, const CUtensorMap& mA, const RdArgs& args,
+                           int grid, cudaStream_t stream) {
+  using L = RdLayout<NT>;
+  auto kern = smallm_rd_kernel<NT>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kDynamic);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = L::kDynamic;
+  cfg.stream = stream;
+  return cudaLaunchKernelEx(&cfg, kern, mC, mX, mA, args);
+}
+
+}  // namespace
+
+size_t small_m_rd_workspace_bytes(int64_t M, int64_t K, int64_t N, int r) {
+  // Sized for the largest grid any device here uses.
+  return rd_plan(M, K, N, r, kMaxGridRd).total;
+}
+
+cudaError_t launch_small_m_rd(const uint16_t* X, const uint8_t* codes, const uint8_t* absmax_q,
+                              const float* absmax_scale, const uint16_t* A, const uint16_t* B, int64_t M, int64_t K,
+                              int64_t N, int r, float scale, uint16_t* Y, float* T_save, void* scratch, int* status,
+                              const Nf4Params& P, cudaStream_t stream) {
+  if (M < 1 || M > kSmallMRdMax || r > 128) return cudaErrorInvalidValue;
+  const RdPlan p = rd_plan(M, K, N, r, rd_sm_count());
+  uint8_t* ws = static_cast<uint8_t*>(scratch);
+  CUtensorMap mC, mX, mA;
+  if (!make_map_2d(&mC, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, K / 2, N, K / 2, 128, kRows,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  // A [K x r] bf16 in tiles of 256 inputs x 64 columns (the A^T row blocks).
+  if (!make_map_2d(&mA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, r, K, static_cast<int64_t>(r) * 2, 64, kKc,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  {
+    // X viewed as [K/64 blocks][2][M tokens][4][8] bf16 (outermost first):
+    // input k = 64 d4 + 16 d1 + 8 d3 + d0 of token d2.
+    const uint64_t dims[5] = {8, 4, static_cast<uint64_t>(M), 2, static_cast<uint64_t>(K / 64)};
+    const uint64_t strides[4] = {32, static_cast<uint64_t>(K) * 2, 16, 128};
+    const uint32_t box[5] = {8, 4, static_cast<uint32_t>(p.MP), 2, 4};
+    if (!make_map_nd(&mX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, 5, dims, strides, box)) return cudaErrorInvalidValue;
+  }
+  // The epilogue asks for the whole shared-memory carveout, as the stream
+  // does: its CTAs then start on an SM as soon as the stream CTA leaves it.
+  static bool carveout_set = false;
+  if (!carveout_set) {
+    cudaFuncSetAttribute(lora_up_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                         cudaSharedmemCarveoutMaxShared);
+    carveout_set = true;
+  }
+
+  RdArgs args{};
+  args.M = static_cast<int>(M);
+  args.N = static_cast<int>(N);
+  args.K = static_cast<int>(K);
+  args.KB = p.KB;
+  args.CH = p.CH;
+  args.RB = p.RB;
+  args.RBW = p.RBW;
+  args.S2 = p.S2;
+  args.U = p.U;
+  args.n_scales = (N * p.KB + 255) / 256;
+  args.absmax_q = absmax_q;
+  args.absmax_scale = absmax_scale;
+  args.partial = reinterpret_cast<float*>(ws + p.off_partial);
+  args.status = status;
+  args.wait_ns = wait_limit_ns();
+  args.nf4 = P;
+  cudaError_t e = p.MP == 8 ? launch_rd_main<1>(mC, mX, mA, args, p.G, stream)
+                            : launch_rd_main<2>(mC, mX, mA, args, p.G, stream);
+  if (e != cudaSuccess) return e;
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>((N + 63) / 64), static_cast<unsigned>((M + 3) / 4), 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1] = {pdl_attribute()};
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  UpArgs ua{};
+  ua.M = static_cast<int>(M);
+  ua.N = static_cast<int>(N);
+  ua.r = r;
+  ua.CH = p.CH;
+  ua.G = p.G;
+  ua.S2 = p.S2;
+  ua.MP = p.MP;
+  ua.RBW = p.RBW;
+  ua.U = p.U;
+  ua.scale = scale;
+  return cudaLaunchKernelEx(&cfg, lora_up_kernel, T_save, B, static_cast<const float*>(args.partial), ua, Y);
+}
+
+}  // namespace qlora
