@@ -79,9 +79,14 @@ struct RdArgs {
   Nf4Params nf4;
 };
 
-__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+// The dynamic shared window of a kernel without static shared memory starts
+// at shared address kSmemBase (after the 1 KB each CTA reserves); the level
+// table sits there, so a table offset formed by one byte permute is the
+// load's register and the base its immediate.
+constexpr uint32_t kSmemBase = 1024;
+__device__ __forceinline__ uint32_t lds32_tab(uint32_t off) {
   uint32_t v;
-  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+  asm volatile("ld.shared.b32 %0, [%1+1024];" : "=r"(v) : "r"(off));
   return v;
 }
 __device__ __forceinline__ uint2 lds64(uint32_t addr) {
@@ -127,7 +132,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* empty = full + kStages;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::offAbort);
   float* lvl2 = reinterpret_cast<float*>(sm + L::offLvl);
-  if (smem_u32(sm) & 1023u) {  // the swizzled copies need a 1024-byte aligned window
+  if (smem_u32(sm) != kSmemBase) {  // table addressing and 1024-byte aligned swizzled copies rely on it
     if (tid == 0 && a.status) atomicCAS(a.status, 0, 0x100 + 62);
     return;
   }
@@ -193,7 +198,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int rg = warp & 7, kh = warp >> 3;
     const int g = lane >> 2, c = lane & 3;
     const uint32_t lane4 = static_cast<uint32_t>(lane) * 4u;
-    const uint32_t tab = smem_u32(sm);
     const uint32_t codes0 = smem_u32(sm + L::offCodes), x0 = smem_u32(sm + L::offX);
     const int KB = a.KB;
     const float mu = centred_mu(a.absmax_scale, a.n_scales, a.nf4.centred);
@@ -351,10 +355,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int t = 0; t < 2; ++t) {
             const uint32_t w0 = s4 < 2 ? w[bb][t][0].x : w[bb][t][0].y;
             const uint32_t w1 = s4 < 2 ? w[bb][t][1].x : w[bb][t][1].y;
-            A[t][0] = lds32(tab + prmt(w0, lane4, 0x5504u | (j0 << 4)));
-            A[t][1] = lds32(tab + prmt(w1, lane4, 0x5504u | (j0 << 4)));
-            A[t][2] = lds32(tab + prmt(w0, lane4, 0x5504u | ((j0 + 1) << 4)));
-            A[t][3] = lds32(tab + prmt(w1, lane4, 0x5504u | ((j0 + 1) << 4)));
+            A[t][0] = lds32_tab(prmt(w0, lane4, 0x5504u | (j0 << 4)));
+            A[t][1] = lds32_tab(prmt(w1, lane4, 0x5504u | (j0 << 4)));
+            A[t][2] = lds32_tab(prmt(w0, lane4, 0x5504u | ((j0 + 1) << 4)));
+            A[t][3] = lds32_tab(prmt(w1, lane4, 0x5504u | ((j0 + 1) << 4)));
           }
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
