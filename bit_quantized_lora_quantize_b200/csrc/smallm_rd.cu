@@ -22,11 +22,11 @@
 //    worked on, with no synchronisation, and the epilogue kernel sums a row
 //    block's partials in a fixed order.
 //
-// T = s X A is computed by the same stream: the rows of A^T are appended to
-// the weight as extra row blocks (bf16, no block constant), so that their
-// products with the X tiles already on chip are partials of T.  A small kernel
-// launched after the stream (programmatic dependent launch) sums the partials
-// into T and Y = bf16(sum of partials + T B).
+// T = s X A is computed by the same stream: the rows of A^T come first as
+// extra row blocks (bf16, no block constant), so that their products with the
+// X tiles already on chip are partials of T, which the last warp of each such
+// row group sums.  A small kernel launched after the stream (programmatic
+// dependent launch) writes Y = bf16(sum of partials + T B).
 //
 // Rounding.  A block's product is sum_k bf16(q_k) x_k (exact products,
 // float32 sums) times the float32 constant a'_b; the other paths multiply by
@@ -68,12 +68,15 @@ struct RdLayout {
 static_assert(RdLayout<2>::kDynamic <= 232448, "shared memory budget");
 
 struct RdArgs {
-  int M, N, K, KB, CH, RB, RBW, S2;
-  int64_t U;             // units = RB * CH; row blocks RBW.. hold the rows of A^T (T = X A)
+  int M, N, K, KB, CH, RB, RBT, S2, r;
+  int64_t U;             // units = RB * CH; row blocks 0 .. RBT-1 hold the rows of A^T (T = X A)
   int64_t n_scales;      // group scales in absmax_scale (the centred mean follows them)
   const uint8_t* absmax_q;
   const float* absmax_scale;
   float* partial;        // [RB][S2][256][MP] float32: one slot per (contributing CTA, block pair)
+  float* T;              // [M x r] float32: T = s X A, finished by the last warp of each A^T row group
+  int* tcnt;             // [RBT][2] arrival counters of those row groups
+  float scale;
   int* status;
   uint64_t wait_ns;
   Nf4Params nf4;
@@ -175,10 +178,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = i % kStages;
         if (i >= kStages && !mbar_wait(&empty[s], ((i / kStages) & 1) ^ 1, ctx)) break;
         mbar_arrive_expect_tx(&full[s], kCodeStage + L::kXStage);
-        if (rb < a.RBW)
-          tma_load_2d(&mapC, &full[s], sm + L::offCodes + s * kCodeStage, ch * 128, rb * kRows);
+        if (rb >= a.RBT)
+          tma_load_2d(&mapC, &full[s], sm + L::offCodes + s * kCodeStage, ch * 128, (rb - a.RBT) * kRows);
         else  // 64 columns of A x 256 inputs, bf16: the same 32 KB
-          tma_load_2d(&mapA, &full[s], sm + L::offCodes + s * kCodeStage, 64 * (rb - a.RBW), ch * kKc);
+          tma_load_2d(&mapA, &full[s], sm + L::offCodes + s * kCodeStage, 64 * rb, ch * kKc);
         tma_load_5d_outer(&mapX, &full[s], sm + L::offX + s * L::kXStage, 4 * ch);
         ++issued;
         if (++ch == CH) {
@@ -209,8 +212,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto fetch = [&](int rbx, int gx, uint4& q, float (&sc)[2]) {
       q = make_uint4(0, 0, 0, 0);
       sc[0] = sc[1] = 0.0f;
-      const int n = rbx * kRows + r_own;
-      if (rbx >= a.RBW || n >= a.N) return;
+      const int n = (rbx - a.RBT) * kRows + r_own;
+      if (rbx < a.RBT || rbx >= a.RB || n >= a.N) return;
       const int64_t b0 = static_cast<int64_t>(n) * KB + 16 * gx;
       if (vec16) {
         q = __ldg(reinterpret_cast<const uint4*>(a.absmax_q + b0));
@@ -256,13 +259,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       {
         const int sb = (ch & 3) * 4 + 2 * kh;
         const uint32_t word = sb < 4 ? gq.x : sb < 8 ? gq.y : sb < 12 ? gq.z : gq.w;
-        const int n = rb * kRows + r_own;
-        const int64_t bl0 = static_cast<int64_t>(n < a.N ? n : 0) * KB + 16 * (ch >> 2);
+        const int n = (rb - a.RBT) * kRows + r_own;  // negative in the A^T row blocks
+        const bool wrow = rb >= a.RBT && n < a.N;
+        const int64_t bl0 = static_cast<int64_t>(wrow ? n : 0) * KB + 16 * (ch >> 2);
 #pragma unroll
         for (int bb = 0; bb < 2; ++bb) {
           const uint32_t q = (word >> (8 * ((sb + bb) & 3))) & 255u;
           const float sc = ((bl0 + sb + bb) >> 8) == (bl0 >> 8) ? gs[0] : gs[1];
-          const bool live = n < a.N && ch * 4 + 2 * kh + bb < KB;
+          const bool live = wrow && ch * 4 + 2 * kh + bb < KB;
           aown[bb] = live ? __fadd_rn(__fmul_rn(lvl2[q], sc), mu) : 0.0f;
         }
       }
@@ -282,36 +286,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!__all_sync(0xFFFFFFFFu, mbar_wait(&full[s], (i / kStages) & 1, ctx))) break;
 
       const uint32_t cs = codes0 + s * kCodeStage, xs = x0 + s * L::kXStage;
-      if (rb >= a.RBW) {
+      if (rb < a.RBT) {
         // Rows of A^T: the stage holds A[256 inputs][64 columns] bf16 with the
-        // 128-byte swizzle; row j of A^T, inputs k..k+3 are 4 scalars of it.
-        // No block constant.  Row groups 0 and 1 cover the 64 columns.
+        // 128-byte swizzle.  One transposing matrix load gives a tile's
+        // fragment: lane i addresses input row k(i) of 8x8 matrix i / 8 (rows
+        // 2c + e <- inputs 16c + 4 s4 + e, +2 for matrices 2 and 3; columns
+        // +8 for matrices 1 and 3), so lane (g, c) receives A^T rows j0 + g
+        // (+8) at exactly the inputs its X fragment holds.  No block
+        // constant.  Row groups 0 and 1 cover the 64 columns.
         if (rg < 2) {
+          const int mq = lane >> 3, ii = lane & 7;
 #pragma unroll
           for (int s4 = 0; s4 < 4; ++s4) {
 #pragma unroll
             for (int bb = 0; bb < 2; ++bb) {
               const int b = 2 * kh + bb;
-              const int k0 = 64 * b + 16 * c + 4 * s4;
+              const int k = 64 * b + 16 * (ii >> 1) + 4 * s4 + (ii & 1) + 2 * (mq >> 1);
               uint32_t A[2][4];
 #pragma unroll
-              for (int t = 0; t < 2; ++t)
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                  const int jj = 32 * rg + 16 * t + 8 * h + g;
-                  uint32_t v[4];
-#pragma unroll
-                  for (int e = 0; e < 4; ++e) {
-                    const int k = k0 + e;
-                    uint16_t x;
-                    asm volatile("ld.shared.u16 %0, [%1];"
-                                 : "=h"(x)
-                                 : "r"(cs + k * 128 + ((((jj >> 3) ^ (k & 7)) & 7) << 4) + (jj & 7) * 2));
-                    v[e] = x;
-                  }
-                  A[t][h] = v[0] | (v[1] << 16);
-                  A[t][h + 2] = v[2] | (v[3] << 16);
-                }
+              for (int t = 0; t < 2; ++t) {
+                const int chunk = 4 * rg + 2 * t + (mq & 1);
+                const uint32_t addr = cs + k * 128 + (((chunk ^ (k & 7)) & 7) << 4);
+                asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(A[t][0]), "=r"(A[t][1]), "=r"(A[t][2]), "=r"(A[t][3])
+                             : "r"(addr));
+              }
 #pragma unroll
               for (int nt = 0; nt < NT; ++nt) {
                 const uint2 xb = lds64(xs + (((b * 2 + (s4 >> 1)) * MP + 8 * nt + g) * 4 + c) * 16 + 8 * (s4 & 1));
@@ -394,18 +393,52 @@ __global__ void __launch_bounds__(kThreads, 1)
         // rg in the slot of (this CTA, block pair); the epilogue kernel sums
         // the slots of each row block in order.
         const int jf = cta_of(static_cast<int64_t>(rb) * CH, a.U, G);
-        if (rb < a.RBW || rg < 2) {
-        float* my = a.partial + ((static_cast<int64_t>(rb) * a.S2 + 2 * (j - jf) + kh) * kRows + 32 * rg) * MP;
+        if (rb >= a.RBT || rg < 2) {
+          const int slot = 2 * (j - jf) + kh;
+          float* my = a.partial + ((static_cast<int64_t>(rb) * a.S2 + slot) * kRows + 32 * rg) * MP;
 #pragma unroll
-        for (int t = 0; t < 2; ++t)
+          for (int t = 0; t < 2; ++t)
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            *reinterpret_cast<float2*>(my + (16 * t + g) * MP + 8 * nt + 2 * c) =
-                make_float2(acc[t][nt][0], acc[t][nt][1]);
-            *reinterpret_cast<float2*>(my + (16 * t + g + 8) * MP + 8 * nt + 2 * c) =
-                make_float2(acc[t][nt][2], acc[t][nt][3]);
+            for (int nt = 0; nt < NT; ++nt) {
+              *reinterpret_cast<float2*>(my + (16 * t + g) * MP + 8 * nt + 2 * c) =
+                  make_float2(acc[t][nt][0], acc[t][nt][1]);
+              *reinterpret_cast<float2*>(my + (16 * t + g + 8) * MP + 8 * nt + 2 * c) =
+                  make_float2(acc[t][nt][2], acc[t][nt][3]);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) acc[t][nt][e] = 0.0f;
+              for (int e = 0; e < 4; ++e) acc[t][nt][e] = 0.0f;
+            }
+          if (rb < a.RBT) {
+            // A row group of A^T: the last of its 2 * (contributing CTAs)
+            // warps sums the slots in order into T (once per call, by the
+            // first CTAs of the grid, early in their ranges).
+            const int jl = cta_of(static_cast<int64_t>(rb + 1) * CH - 1, a.U, G);
+            const int nparts = 2 * (jl - jf + 1);
+            __threadfence();
+            __syncwarp();
+            int old = 0;
+            if (lane == 0) old = atomicAdd(a.tcnt + rb * 2 + rg, 1);
+            old = __shfl_sync(0xFFFFFFFFu, old, 0);
+            if (old == nparts - 1) {
+              __threadfence();
+              const float* base = a.partial + (static_cast<int64_t>(rb) * a.S2 * kRows + 32 * rg) * MP;
+#pragma unroll
+              for (int t = 0; t < 2; ++t)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                  const int row = 16 * t + 8 * h + g, col = 64 * rb + 32 * rg + row;
+#pragma unroll
+                  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                      const int m = 8 * nt + 2 * c + e;
+                      float v = 0.0f;
+                      for (int p = 0; p < nparts; ++p)
+                        v += __ldcg(base + (static_cast<int64_t>(p) * kRows + row) * MP + m);
+                      if (m < a.M && col < a.r) a.T[static_cast<int64_t>(m) * a.r + col] = __fmul_rn(a.scale, v);
+                    }
+                }
+              if (lane == 0) a.tcnt[rb * 2 + rg] = 0;
+            }
           }
         }
       }
@@ -421,22 +454,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ranks q r/8 .. (q + 1) r/8 - 1 of T B, then a fixed butterfly over the 8
 // slices completes the sum.
 struct UpArgs {
-  int M, N, r, CH, G, S2, MP, RBW;
+  int M, N, r, CH, G, S2, MP, RBT;
   int64_t U;
-  float scale;
 };
 
-// Sum, in slot order, the partials of row `row` of row block rb for token m.
-__device__ __forceinline__ float sum_partials(const float* partial, const UpArgs& u, int rb, int row, int m) {
-  const int jf = cta_of(static_cast<int64_t>(rb) * u.CH, u.U, u.G);
-  const int jl = cta_of(static_cast<int64_t>(rb + 1) * u.CH - 1, u.U, u.G);
-  float v = 0.0f;
-  for (int p = 0; p < 2 * (jl - jf + 1); ++p)
-    v += __ldcg(partial + ((static_cast<int64_t>(rb) * u.S2 + p) * kRows + row) * u.MP + m);
-  return v;
-}
-
-__global__ void __launch_bounds__(256) lora_up_kernel(float* __restrict__ T, const uint16_t* __restrict__ B,
+__global__ void __launch_bounds__(256) lora_up_kernel(const float* __restrict__ T, const uint16_t* __restrict__ B,
                                                       const float* __restrict__ partial, const UpArgs u,
                                                       uint16_t* __restrict__ Y) {
   const int lane = threadIdx.x & 31, q = lane & 7, p = lane >> 3;
@@ -449,25 +471,19 @@ __global__ void __launch_bounds__(256) lora_up_kernel(float* __restrict__ T, con
 #pragma unroll
   for (int e = 0; e < 16; ++e)
     bw[e] = live && e < rs ? __ldg(reinterpret_cast<const uint32_t*>(B + static_cast<int64_t>(q * rs + e) * u.N + n)) : 0u;
-  griddep_wait();  // the weight stream has completed
-  // This CTA's four rows of T = s X A, summed from the A^T row blocks'
-  // partials (the CTAs of the first column also store T for the backward);
-  // the partial slots of Y are read in the same round.
+  griddep_wait();  // the weight stream (which also finished T) has completed
+  // This CTA's four rows of T, staged once; the partial slots of Y are read
+  // in the same round.
   __shared__ float Ts[4][128];
   for (int i = threadIdx.x; i < 4 * u.r; i += blockDim.x) {
     const int mm = i / u.r, jj = i % u.r;
-    float t = 0.0f;
-    if (m0 + mm < u.M) {
-      t = __fmul_rn(u.scale, sum_partials(partial, u, u.RBW + jj / 64, jj % 64, m0 + mm));
-      if (blockIdx.x == 0) T[static_cast<int64_t>(m0 + mm) * u.r + jj] = t;
-    }
-    Ts[mm][jj] = t;
+    Ts[mm][jj] = m0 + mm < u.M ? __ldcg(T + static_cast<int64_t>(m0 + mm) * u.r + jj) : 0.0f;
   }
   float z[4][2];
 #pragma unroll
   for (int mm = 0; mm < 4; ++mm) z[mm][0] = z[mm][1] = 0.0f;
   if (live) {
-    const int rb = n / kRows, row = n % kRows;
+    const int rb = u.RBT + n / kRows, row = n % kRows;
     const int jf = cta_of(static_cast<int64_t>(rb) * u.CH, u.U, u.G);
     const int jl = cta_of(static_cast<int64_t>(rb + 1) * u.CH - 1, u.U, u.G);
     const int nparts = 2 * (jl - jf + 1);
@@ -522,9 +538,9 @@ int rd_sm_count() {
 }
 
 struct RdPlan {
-  int KB, CH, RB, RBW, G, S2, MP;
+  int KB, CH, RB, RBT, G, S2, MP;
   int64_t U;
-  size_t off_partial, total;
+  size_t off_partial, off_tcnt, total;
 };
 
 size_t r256(size_t x) { return (x + 255) / 256 * 256; }
@@ -533,8 +549,8 @@ RdPlan rd_plan(int64_t M, int64_t K, int64_t N, int r, int sms) {
   RdPlan p{};
   p.KB = static_cast<int>(K / 64);
   p.CH = static_cast<int>((K + kKc - 1) / kKc);
-  p.RBW = static_cast<int>((N + kRows - 1) / kRows);
-  p.RB = p.RBW + (r + 63) / 64;  // + the rows of A^T, 64 per block
+  p.RBT = (r + 63) / 64;  // the rows of A^T, 64 per block, first
+  p.RB = p.RBT + static_cast<int>((N + kRows - 1) / kRows);
   p.U = static_cast<int64_t>(p.RB) * p.CH;
   p.G = static_cast<int>(std::min<int64_t>({static_cast<int64_t>(sms), static_cast<int64_t>(kMaxGridRd), p.U}));
   // A row block spans at most ceil(CH / (U / G)) + 1 CTAs.
@@ -545,6 +561,8 @@ RdPlan rd_plan(int64_t M, int64_t K, int64_t N, int r, int sms) {
   size_t o = 0;
   p.off_partial = o;
   o += r256(static_cast<size_t>(p.RB) * p.S2 * kRows * p.MP * 4);
+  p.off_tcnt = o;
+  o += r256(static_cast<size_t>(p.RBT) * 2 * 4);
   p.total = o;
   return p;
 }
@@ -610,7 +628,11 @@ cudaError_t launch_small_m_rd(const uint16_t* X, const uint8_t* codes, const uin
   args.KB = p.KB;
   args.CH = p.CH;
   args.RB = p.RB;
-  args.RBW = p.RBW;
+  args.RBT = p.RBT;
+  args.r = r;
+  args.T = T_save;
+  args.tcnt = reinterpret_cast<int*>(ws + p.off_tcnt);
+  args.scale = scale;
   args.S2 = p.S2;
   args.U = p.U;
   args.n_scales = (N * p.KB + 255) / 256;
@@ -639,10 +661,10 @@ cudaError_t launch_small_m_rd(const uint16_t* X, const uint8_t* codes, const uin
   ua.G = p.G;
   ua.S2 = p.S2;
   ua.MP = p.MP;
-  ua.RBW = p.RBW;
+  ua.RBT = p.RBT;
   ua.U = p.U;
-  ua.scale = scale;
-  return cudaLaunchKernelEx(&cfg, lora_up_kernel, T_save, B, static_cast<const float*>(args.partial), ua, Y);
+  return cudaLaunchKernelEx(&cfg, lora_up_kernel, static_cast<const float*>(T_save), B,
+                            static_cast<const float*>(args.partial), ua, Y);
 }
 
 }  // namespace qlora
