@@ -204,9 +204,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t codes0 = smem_u32(sm + L::offCodes), x0 = smem_u32(sm + L::offX);
     const int KB = a.KB;
     const float mu = centred_mu(a.absmax_scale, a.n_scales, a.nf4.centred);
-    // This lane loads the constants of row r_own (t = c >> 1, h = c & 1) and
-    // hands them to the lanes that need them.
-    const int r_own = 32 * rg + 16 * (c >> 1) + 8 * (c & 1) + g;
+    // Weight rows of a 16-row tile: fragment row g is row 2g, fragment row
+    // g + 8 is row 2g + 1.  The 16 lanes of a half-warp then read their code
+    // bytes from 8 different 16-byte chunk positions of the 128-byte-swizzled
+    // tile (no bank conflict).  This lane loads the constants of row r_own
+    // (t = c >> 1, h = c & 1) and hands them to the lanes that need them.
+    const int r_own = 32 * rg + 16 * (c >> 1) + 2 * g + (c & 1);
     const bool vec16 = (KB & 15) == 0 && (reinterpret_cast<uintptr_t>(a.absmax_q) & 15u) == 0;
     // Raw 8-bit constants and the two group scales of 16 consecutive blocks.
     auto fetch = [&](int rbx, int gx, uint4& q, float (&sc)[2]) {
@@ -337,8 +340,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = 0; t < 2; ++t)
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            const int r = 32 * rg + 16 * t + 8 * h + g, b = 2 * kh + bb;
-            w[bb][t][h] = lds64(cs + r * 128 + (((2 * b + (c >> 1)) ^ g) << 4) + 8 * (c & 1));
+            const int r = 32 * rg + 16 * t + 2 * g + h, b = 2 * kh + bb;
+            w[bb][t][h] = lds64(cs + r * 128 + ((((2 * b + (c >> 1)) ^ r) & 7) << 4) + 8 * (c & 1));
           }
       float bl[2][2][NT][4];  // [bb][t][nt]
 #pragma unroll
@@ -396,13 +399,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (rb >= a.RBT || rg < 2) {
           const int slot = 2 * (j - jf) + kh;
           float* my = a.partial + ((static_cast<int64_t>(rb) * a.S2 + slot) * kRows + 32 * rg) * MP;
+          // Rows of fragment rows g and g + 8 (A^T tiles keep the plain order).
+          const bool tb = rb < a.RBT;
+          const int r0 = tb ? g : 2 * g, r1 = tb ? g + 8 : 2 * g + 1;
 #pragma unroll
           for (int t = 0; t < 2; ++t)
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-              *reinterpret_cast<float2*>(my + (16 * t + g) * MP + 8 * nt + 2 * c) =
+              *reinterpret_cast<float2*>(my + (16 * t + r0) * MP + 8 * nt + 2 * c) =
                   make_float2(acc[t][nt][0], acc[t][nt][1]);
-              *reinterpret_cast<float2*>(my + (16 * t + g + 8) * MP + 8 * nt + 2 * c) =
+              *reinterpret_cast<float2*>(my + (16 * t + r1) * MP + 8 * nt + 2 * c) =
                   make_float2(acc[t][nt][2], acc[t][nt][3]);
 #pragma unroll
               for (int e = 0; e < 4; ++e) acc[t][nt][e] = 0.0f;
