@@ -694,7 +694,8 @@ def bench_paged_adamw(args, lins, bucket, dev, flush, peaks):
     return {"params": opt.n, "state_bytes": opt.state_bytes, "us_per_step": us, "gbs": gbs,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / peaks["hbm_gbs"], "bytes_per_step": by,
-                         "bytes_counted": "30 B per parameter (16 read, 14 written)"},
+                         "bytes_counted": "30 B per parameter (16 read, 14 written)",
+                         "traffic": traffic_for("adamw_step/block")},
             "us_per_step_after_eviction": us_paged,
             "note": "after eviction: prefetch of the 3 state vectors host->GPU plus the step, device time"}
 
