@@ -173,13 +173,20 @@ QLORA_API qlora_status qlora_dequantize_4bit(const uint8_t* codes, const uint8_t
  * that are not multiples of 8 run with A, B, T_save, dA and dB padded with
  * zeros to the next multiple of 8 inside the workspace (a few small copy
  * kernels around the GEMM); ranks above 128 always take the pair GEMMs.
- * The forward is one kernel launch.  For M <= 128 its thread blocks wait
- * for one another (cooperative launch: all of them must be resident at
- * once); if the device cannot hold them next to other work the call returns
- * QLORA_ERR_CUDA and launches nothing.  For larger M, blocks that finished
- * T for a 512-row block release the output tiles of those rows (work is
- * handed out in that order, so no residency is needed).  Sums are taken in a
- * fixed order: results are bit-reproducible run to run.
+ * For up to 8 tokens (up to 16 when N*K >= 2^27) the forward is two
+ * launches chained by programmatic dependent launch: a weight stream that
+ * also forms T, and a small kernel that sums its partials and adds T B;
+ * neither needs its blocks to be resident together.  On this path the block
+ * constant multiplies each 64-input block's partial product (bf16 level
+ * times x, float32 sums) rather than each weight; either way a term carries
+ * one bf16 rounding.  For other M <= 128 the forward is one launch whose
+ * thread blocks wait for one another (cooperative launch: all of them must
+ * be resident at once); if the device cannot hold them next to other work
+ * the call returns QLORA_ERR_CUDA and launches nothing.  For larger M it is
+ * one launch in which blocks that finished T for a 512-row block release
+ * the output tiles of those rows (work is handed out in that order, so no
+ * residency is needed).  Sums are taken in a fixed order: results are
+ * bit-reproducible run to run.
  */
 QLORA_API qlora_status qlora_linear_fwd(const uint16_t* X, int64_t M, int64_t K, int64_t N, const uint8_t* codes,
                               const uint8_t* absmax_q, const float* absmax_scale, const uint16_t* A,
