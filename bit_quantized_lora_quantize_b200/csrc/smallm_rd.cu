@@ -376,16 +376,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      // Block constant times the block's partial product, two accumulators
+      // (same row, two tokens) per packed float32 multiply-add.
 #pragma unroll
       for (int bb = 0; bb < 2; ++bb)
 #pragma unroll
         for (int t = 0; t < 2; ++t)
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
-            acc[t][nt][0] = fmaf(av[t][0][bb], bl[bb][t][nt][0], acc[t][nt][0]);
-            acc[t][nt][1] = fmaf(av[t][0][bb], bl[bb][t][nt][1], acc[t][nt][1]);
-            acc[t][nt][2] = fmaf(av[t][1][bb], bl[bb][t][nt][2], acc[t][nt][2]);
-            acc[t][nt][3] = fmaf(av[t][1][bb], bl[bb][t][nt][3], acc[t][nt][3]);
+            const float2 a0 = make_float2(av[t][0][bb], av[t][0][bb]);
+            const float2 a1 = make_float2(av[t][1][bb], av[t][1][bb]);
+            const float2 r0 = __ffma2_rn(a0, make_float2(bl[bb][t][nt][0], bl[bb][t][nt][1]),
+                                         make_float2(acc[t][nt][0], acc[t][nt][1]));
+            const float2 r1 = __ffma2_rn(a1, make_float2(bl[bb][t][nt][2], bl[bb][t][nt][3]),
+                                         make_float2(acc[t][nt][2], acc[t][nt][3]));
+            acc[t][nt][0] = r0.x;
+            acc[t][nt][1] = r0.y;
+            acc[t][nt][2] = r1.x;
+            acc[t][nt][3] = r1.y;
           }
       }
       __syncwarp();
