@@ -874,15 +874,22 @@ def bench_tiny(args, q, synthetic, dev, flush, iters=50):
 # ---------------------------------------------------------------- small-M sweep
 def small_m_sweep(q, synthetic, dev, flush, iters=10):
     """Small-M forward (W [N x 8192] NF4, M tokens, r = 64): NF4 weight bytes
-    streamed per second, L2 flushed before every timed call."""
+    streamed per second, L2 flushed before every timed call (`us`).  Also
+    `us_back_to_back`: calls on four different weights in turn (4 x 34.6 MB
+    or 4 x 93 MB, more than L2, so every call still reads its weight from
+    HBM) between one pair of events, per call -- what a decode loop over
+    layers sees, without one event pair's launch latency per call."""
     import torch
 
     peaks = load_peaks()
     out = []
     for N in (8192, 22016):
-        W = synthetic.weight_only(N, 8192, seed=4).to(dev)
-        Wp = q.qlora_quantize_nf4(W)
-        del W
+        Wps = []
+        for i in range(4):
+            W = synthetic.weight_only(N, 8192, seed=4 + i).to(dev)
+            Wps.append(q.qlora_quantize_nf4(W))
+            del W
+        Wp = Wps[0]
         nb = nf4_bytes(N * 8192)
         for M in (1, 4, 16, 64):
             case = synthetic.small_m_case(M, N)
@@ -902,8 +909,19 @@ def small_m_sweep(q, synthetic, dev, flush, iters=10):
             torch.cuda.synchronize()
             us = sorted(a.elapsed_time(b) * 1e3 for a, b in evs)[iters // 2]
             gbs = nb / (us * 1e-6) / 1e9
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            flush.zero_()
+            e0.record(stream)
+            for _ in range(iters):
+                for w in Wps:
+                    q.qlora_linear_fwd(X, w, A, B, 0.25, workspace=ws, Y=Y, T_save=T)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            us_b2b = e0.elapsed_time(e1) * 1e3 / (iters * len(Wps))
             out.append({"N": N, "K": 8192, "M": M, "us": us, "nf4_weight_gbs": gbs,
                         "frac_hbm": gbs / peaks["hbm_gbs"], "nf4_bytes": nb,
+                        "us_back_to_back": us_b2b,
+                        "frac_hbm_back_to_back": nb / (us_b2b * 1e-6) / 1e9 / peaks["hbm_gbs"],
                         "kernel": "small_m_nf4_fwd" if M <= 128 else "fused_nf4_fwd"})
             if q.qlora_check_status(ws) != 0:
                 raise RuntimeError("device pipeline timeout (small M)")
