@@ -82,7 +82,7 @@ def test_traffic_entry_goes_null_when_the_kernel_source_changes(tmp_path, monkey
 
 def test_reference_arm_prints_the_contract_line():
     """`bench.py --impl reference` times the oracle on the host cores and
-    prints one JSON line with the keys the driver reads."""
+    prints one JSON line with the keys of the bench contract."""
     import json
     import pathlib
     import subprocess
