@@ -84,11 +84,13 @@ def bf16_values(rng, n, std):
     return bf16_round(rng.standard_normal(n).astype(np.float32) * np.float32(std))
 
 
-@pytest.mark.parametrize("code", ["nf4", "fp4", "int4"])
-@pytest.mark.parametrize("n", [1, 2, 63, 64, 65, 127, 130, 64 * 256 + 5])
+# NF4 on every size; the other codebooks on a subset of them.
+BRUTE_CASES = ([("nf4", n) for n in (1, 2, 63, 64, 65, 127, 130, 64 * 256 + 5)]
+               + [(c, n) for c in ("fp4", "int4") for n in (1, 65, 64 * 256 + 5)])
+
+
+@pytest.mark.parametrize("code,n", BRUTE_CASES)
 def test_quantize_matches_brute_force(n, code):
-    if code != "nf4" and n not in (1, 65, 64 * 256 + 5):
-        pytest.skip("the other codebooks on a subset of the sizes")
     rng = np.random.default_rng(100 + n)
     x = bf16_values(rng, n, 0.02)
     if n > 70:
