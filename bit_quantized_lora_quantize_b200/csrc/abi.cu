@@ -155,6 +155,28 @@ qlora_status check_linear_shape(int64_t M, int64_t K, int64_t N, int32_t r) {
 
 uint64_t wait_limit_ns() { return g_wait_ns.load(std::memory_order_relaxed); }
 
+namespace {
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_sm_count[kMaxDevices];
+std::atomic<int> g_l2_bytes[kMaxDevices];
+
+// Attribute `what` of the current device, read once per device; `fallback`
+// when the device or the attribute cannot be read.
+int cached_attribute(std::atomic<int>* cache, cudaDeviceAttr what, int fallback) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return fallback;
+  int v = dev < kMaxDevices ? cache[dev].load(std::memory_order_relaxed) : 0;
+  if (v > 0) return v;
+  if (cudaDeviceGetAttribute(&v, what, dev) != cudaSuccess || v <= 0) return fallback;
+  if (dev < kMaxDevices) cache[dev].store(v, std::memory_order_relaxed);
+  return v;
+}
+}  // namespace
+
+int device_sm_count() { return cached_attribute(g_sm_count, cudaDevAttrMultiProcessorCount, 148); }
+
+int device_l2_bytes() { return cached_attribute(g_l2_bytes, cudaDevAttrL2CacheSize, 126 << 20); }
+
 ProfScope::ProfScope(cudaStream_t s, const char* n, int l) : on(false), st(s), name(n), launches(l) {
   std::lock_guard<std::mutex> g(g_prof_mu);
   on = g_prof_on;

@@ -94,10 +94,8 @@ __global__ void __launch_bounds__(kAdamThreads) adamw_kernel(float* __restrict__
 }
 
 int adam_grid(int64_t work) {
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t want = (work + kAdamThreads - 1) / kAdamThreads;
-  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, static_cast<int64_t>(sms > 0 ? sms : 148) * 8)));
+  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, static_cast<int64_t>(device_sm_count()) * 8)));
 }
 
 }  // namespace

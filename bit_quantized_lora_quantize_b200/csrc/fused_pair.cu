@@ -777,23 +777,11 @@ cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& c, const CUtens
   return cudaLaunchKernelEx(&cfg, kern, a, c, a2, b2, abs, rmap, tmaps, args);
 }
 
-int l2_bytes() {
-  static int cached[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 126 << 20;
-  if (!cached[dev]) {
-    int v = 0;
-    cudaDeviceGetAttribute(&v, cudaDevAttrL2CacheSize, dev);
-    cached[dev] = v > 0 ? v : (126 << 20);
-  }
-  return cached[dev];
-}
-
 // Row blocks per tile group: as few groups as keep one group's activation
 // rows (512 x depth bf16 per row block) within half of L2, balanced.
 int group_rows_for(int tiles_m, int64_t depth) {
   const int64_t block_bytes = static_cast<int64_t>(kPairRows) * depth * 2;
-  const int64_t budget = l2_bytes() / 2;
+  const int64_t budget = device_l2_bytes() / 2;
   const int64_t fit = std::max<int64_t>(1, budget / std::max<int64_t>(1, block_bytes));
   const int64_t groups = (tiles_m + fit - 1) / fit;
   return static_cast<int>((tiles_m + groups - 1) / groups);
@@ -822,12 +810,7 @@ void plan_units(PairArgs& args, int64_t M, int64_t cols, int64_t depth, int r, f
 }
 
 // CTA pairs resident at once (one 1-CTA-per-SM pair per two SMs).
-int resident_pairs() {
-  int dev = 0, sms = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-    return 1;
-  return std::max(1, sms / 2);
-}
+int resident_pairs() { return std::max(1, device_sm_count() / 2); }
 
 }  // namespace
 

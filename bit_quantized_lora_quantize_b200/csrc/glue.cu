@@ -88,10 +88,8 @@ __global__ void __launch_bounds__(kGlueThreads) silu_gate_bwd_kernel(
 }
 
 int glue_grid(int64_t n8) {
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t want = (n8 + kGlueThreads - 1) / kGlueThreads;
-  const int64_t cap = static_cast<int64_t>(sms > 0 ? sms : 148) * 8;  // 8 resident CTAs of 256 per SM
+  const int64_t cap = static_cast<int64_t>(device_sm_count()) * 8;  // 8 resident CTAs of 256 per SM
   return static_cast<int>(std::max<int64_t>(1, std::min(want, cap)));
 }
 

@@ -15,6 +15,12 @@ namespace qlora {
 constexpr uint64_t kMaxWaitTimeoutNs = 60000000000ull;  // 60 s
 uint64_t wait_limit_ns();
 
+// Multiprocessor count and L2 size of the current device, read once per
+// device (148 SMs and 126 MB when they cannot be read).  Safe to call from
+// several host threads.
+int device_sm_count();
+int device_l2_bytes();
+
 // Status words the library keeps on the device for calls without a
 // workspace: each reads the current device's word (after the stream's work),
 // clears it if it was set and returns it in *word.

@@ -400,13 +400,7 @@ cudaError_t launch_quantize_nf4(const uint16_t* W, int64_t numel, uint8_t* codes
   if (!make_map_2d(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, kBlock, full_rows > 0 ? full_rows : 1, kBlock * 2,
                    kBlock, kGroup, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  static int sm_count = 0;
-  if (sm_count == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (cudaDeviceGetAttribute(&sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sm_count <= 0)
-      sm_count = 148;
-  }
+  const int sm_count = device_sm_count();
   cudaError_t e = cudaFuncSetAttribute(quantize_nf4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kQuantSmem);
   if (e != cudaSuccess) return e;
   if (P.centred) {

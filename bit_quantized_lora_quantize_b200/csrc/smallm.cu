@@ -761,18 +761,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-int sm_count() {
-  static int cached[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (!cached[dev]) {
-    int v = 0;
-    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
-    cached[dev] = v > 0 ? v : 148;
-  }
-  return cached[dev];
-}
-
 template <int MP>
 cudaError_t launch_mp(const CUtensorMap& c, const CUtensorMap& x, const CUtensorMap& a, const CUtensorMap& b,
                       const CUtensorMap& t, const SmallMArgs& args, cudaStream_t stream) {
@@ -849,7 +837,7 @@ cudaError_t launch_small_m_fwd(const uint16_t* X, const uint8_t* codes, const ui
   a.L = 2 * rp / 64;
   a.tiles = static_cast<int>((N + kTileRows - 1) / kTileRows);
   a.W = static_cast<int64_t>(a.KB) * (a.tiles + 1);
-  a.grid = static_cast<int>(std::min<int64_t>({static_cast<int64_t>(sm_count()), static_cast<int64_t>(kMaxGrid),
+  a.grid = static_cast<int>(std::min<int64_t>({static_cast<int64_t>(device_sm_count()), static_cast<int64_t>(kMaxGrid),
                                                std::max<int64_t>(1, a.W / 8)}));
   a.nT = std::min(a.grid, std::max(1, (a.KB + 1) / 2));
   // Every CTA's range must cover its T units; otherwise run on one CTA.

@@ -33,6 +33,7 @@
 // the dequantized weight bf16(fp32(q_k) a'_b).  Each form carries one bf16
 // rounding of relative size <= 2^-9 per term against the exact q_k a'_b x_k.
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -539,18 +540,6 @@ __global__ void __launch_bounds__(256) lora_up_kernel(const float* __restrict__ 
   }
 }
 
-int rd_sm_count() {
-  static int cached[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (!cached[dev]) {
-    int v = 0;
-    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
-    cached[dev] = v > 0 ? v : 148;
-  }
-  return cached[dev];
-}
-
 struct RdPlan {
   int KB, CH, RB, RBT, G, S2, MP;
   int64_t U;
@@ -608,7 +597,7 @@ cudaError_t launch_small_m_rd(const uint16_t* X, const uint8_t* codes, const uin
                               int64_t N, int r, float scale, uint16_t* Y, float* T_save, void* scratch, int* status,
                               const Nf4Params& P, cudaStream_t stream) {
   if (M < 1 || M > kSmallMRdMax || r > 128) return cudaErrorInvalidValue;
-  const RdPlan p = rd_plan(M, K, N, r, rd_sm_count());
+  const RdPlan p = rd_plan(M, K, N, r, device_sm_count());
   uint8_t* ws = static_cast<uint8_t*>(scratch);
   CUtensorMap mC, mX, mA;
   if (!make_map_2d(&mC, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, K / 2, N, K / 2, 128, kRows,
@@ -628,11 +617,19 @@ cudaError_t launch_small_m_rd(const uint16_t* X, const uint8_t* codes, const uin
   }
   // The epilogue asks for the whole shared-memory carveout, as the stream
   // does: its CTAs then start on an SM as soon as the stream CTA leaves it.
-  static bool carveout_set = false;
-  if (!carveout_set) {
-    cudaFuncSetAttribute(lora_up_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                         cudaSharedmemCarveoutMaxShared);
-    carveout_set = true;
+  // A preference, set once per device (a failure only costs that overlap).
+  {
+    static std::atomic<uint64_t> carveout_set{0};
+    int dev = 0;
+    const bool known = cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64;
+    const uint64_t bit = known ? (uint64_t(1) << dev) : 0;
+    if (!known || !(carveout_set.load(std::memory_order_relaxed) & bit)) {
+      if (cudaFuncSetAttribute(lora_up_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               cudaSharedmemCarveoutMaxShared) == cudaSuccess)
+        carveout_set.fetch_or(bit, std::memory_order_relaxed);
+      else
+        cudaGetLastError();  // the preference is optional: drop its recorded error
+    }
   }
 
   RdArgs args{};
