@@ -872,25 +872,36 @@ def bench_tiny(args, q, synthetic, dev, flush, iters=50):
 
 
 # ---------------------------------------------------------------- small-M sweep
+def weight_copies(Wp, nbytes, l2_bytes, at_least=4):
+    """Wp and clones of it at distinct addresses, together at least three
+    times the L2 size, so that a weight used once per rotation has left L2
+    before its next use (L2 lines are physical: equal contents do not share)."""
+    import dataclasses
+
+    n = max(at_least, -(-3 * l2_bytes // nbytes))
+    return [Wp] + [dataclasses.replace(Wp, codes=Wp.codes.clone(), absmax_q=Wp.absmax_q.clone(),
+                                       absmax_scale=Wp.absmax_scale.clone()) for _ in range(n - 1)]
+
+
 def small_m_sweep(q, synthetic, dev, flush, iters=10):
     """Small-M forward (W [N x 8192] NF4, M tokens, r = 64): NF4 weight bytes
     streamed per second, L2 flushed before every timed call (`us`).  Also
-    `us_back_to_back`: calls on four different weights in turn (4 x 34.6 MB
-    or 4 x 93 MB, more than L2, so every call still reads its weight from
-    HBM) between one pair of events, per call -- what a decode loop over
-    layers sees, without one event pair's launch latency per call."""
+    `us_back_to_back`: calls on copies of the weight in turn, at least three
+    times the L2 size in all (12 x 34.6 MB or 5 x 93 MB on B200), so that
+    each call reads its weight from HBM, between one pair of events, per
+    call -- what a decode loop over layers sees, without one event pair's
+    launch latency per call."""
     import torch
 
     peaks = load_peaks()
+    l2 = getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 0) or (126 << 20)
     out = []
     for N in (8192, 22016):
-        Wps = []
-        for i in range(4):
-            W = synthetic.weight_only(N, 8192, seed=4 + i).to(dev)
-            Wps.append(q.qlora_quantize_nf4(W))
-            del W
-        Wp = Wps[0]
+        W = synthetic.weight_only(N, 8192, seed=4).to(dev)
+        Wp = q.qlora_quantize_nf4(W)
+        del W
         nb = nf4_bytes(N * 8192)
+        Wps = weight_copies(Wp, nb, l2)
         for M in (1, 4, 16, 64):
             case = synthetic.small_m_case(M, N)
             X, A, B = (t.to(dev) for t in (case.X, case.A, case.B))
@@ -920,7 +931,7 @@ def small_m_sweep(q, synthetic, dev, flush, iters=10):
             us_b2b = e0.elapsed_time(e1) * 1e3 / (iters * len(Wps))
             out.append({"N": N, "K": 8192, "M": M, "us": us, "nf4_weight_gbs": gbs,
                         "frac_hbm": gbs / peaks["hbm_gbs"], "nf4_bytes": nb,
-                        "us_back_to_back": us_b2b,
+                        "us_back_to_back": us_b2b, "back_to_back_copies": len(Wps),
                         "frac_hbm_back_to_back": nb / (us_b2b * 1e-6) / 1e9 / peaks["hbm_gbs"],
                         "kernel": "small_m_nf4_fwd" if M <= 128 else "fused_nf4_fwd"})
             if q.qlora_check_status(ws) != 0:

@@ -1,8 +1,9 @@
 """Host-side logic of bench.py that needs no GPU: the clock sampler (run
 against a fake NVML module in the child process it starts), the rule that
 keeps a committed DRAM-traffic figure only while its kernel's sources are
-unchanged, the oracle reference arm's JSON line, and the multi-GPU launch
-(re-execution under torchrun, world-size check)."""
+unchanged, the oracle reference arm's JSON line, the multi-GPU launch
+(re-execution under torchrun, world-size check), and the weight copies the
+small-M back-to-back timing rotates over."""
 import sys
 import time
 
@@ -120,3 +121,35 @@ def test_world_size_must_match_gpus(monkeypatch):
     monkeypatch.setenv("RANK", "0")
     with pytest.raises(SystemExit):
         bench.main(["--gpus", "4"])
+
+
+def test_back_to_back_weight_copies_exceed_three_l2():
+    """The small-M back-to-back timing rotates over clones of one packed
+    weight: at least four, together at least three times the L2 size, each
+    in its own storage with the same contents."""
+    import torch
+
+    import bench
+    from bit_quantized_lora_quantize_b200.qlora import PackedNF4, packed_sizes
+
+    l2 = 126 << 20
+    for N in (8192, 22016):
+        numel = N * 8192
+        nc, nb, ng = packed_sizes(numel)
+        Wp = PackedNF4(torch.randint(0, 256, (nc,), dtype=torch.uint8), torch.randint(0, 256, (nb,), dtype=torch.uint8),
+                       torch.rand(ng), (N, 8192))
+        nbytes = bench.nf4_bytes(numel)
+        assert nbytes == nc + nb + 4 * ng
+        ws = bench.weight_copies(Wp, nbytes, l2)
+        assert len(ws) >= 4 and len(ws) * nbytes >= 3 * l2
+        assert len(ws) == 4 or (len(ws) - 1) * nbytes < 3 * l2  # no more copies than needed
+        assert ws[0] is Wp
+        ptrs = {w.codes.data_ptr() for w in ws} | {w.absmax_q.data_ptr() for w in ws} | \
+               {w.absmax_scale.data_ptr() for w in ws}
+        assert len(ptrs) == 3 * len(ws)
+        for w in ws[1:]:
+            assert torch.equal(w.codes, Wp.codes) and torch.equal(w.absmax_q, Wp.absmax_q)
+            assert torch.equal(w.absmax_scale, Wp.absmax_scale)
+            assert (w.shape, w.code, w.dq) == (Wp.shape, Wp.code, Wp.dq)
+    assert len(bench.weight_copies(Wp, bench.nf4_bytes(8192 * 8192), l2)) == 12
+    assert len(bench.weight_copies(Wp, bench.nf4_bytes(22016 * 8192), l2)) == 5
