@@ -129,7 +129,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   using L = RdLayout<NT>;
   constexpr int MP = L::MP;
   // The kernel has no static shared memory: the dynamic window starts at
-  // shared address 0, aligned for the 128-byte-swizzled TMA tiles.
+  // shared address kSmemBase, aligned for the 128-byte-swizzled TMA tiles.
   extern __shared__ __align__(1024) uint8_t sm[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + L::offBar);
