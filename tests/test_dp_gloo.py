@@ -4,6 +4,7 @@ views of one gradient bucket (the structure the benchmark's backward writes
 into), sum the bucket with its all-reduce, and must reproduce the full-batch
 gradients."""
 
+import datetime
 import os
 import socket
 
@@ -30,7 +31,7 @@ def _rank_main(rank, world, port, out):
 
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
-    dist.init_process_group("gloo", rank=rank, world_size=world)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
     try:
         # Two linears of different shapes share one bucket, as the block
         # step's seven linears do.
@@ -77,7 +78,9 @@ def test_shard_rows_cover_all_tokens():
 
 def test_two_rank_gradient_sum_equals_full_batch():
     port = _free_port()
-    with mp.Manager() as m:
+    # The result dict's server process is spawned like the ranks: forking a
+    # process that already runs threads can deadlock the child.
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.spawn(_rank_main, args=(2, port, out), nprocs=2, join=True)
         assert len(out["errs"]) == 4 and max(out["errs"]) < 1e-5, out["errs"]
