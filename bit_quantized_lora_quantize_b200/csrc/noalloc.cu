@@ -21,6 +21,7 @@
 // without ordering) race on it.  The first 256 bytes hold the status word: a
 // pipeline wait that gave up sets it, and qlora_check_status reports and
 // clears it (calls leave it alone, so a timeout stays visible until then).
+#include <cmath>
 #include <cstdint>
 #include <mutex>
 
@@ -94,7 +95,7 @@ extern "C" qlora_status qlora_linear_fwd_noalloc(const uint16_t* X, int64_t M, i
                                                  const float* absmax_scale, const uint16_t* A, const uint16_t* B,
                                                  int32_t r, float scale, uint16_t* Y, float* T_save, void* stream) {
   if (!X || !codes || !absmax_q || !absmax_scale || !A || !B || !Y || !T_save) return QLORA_ERR_INVALID_ARG;
-  if (!(scale == scale) || scale - scale != 0.0f) return QLORA_ERR_INVALID_ARG;  // NaN or infinite
+  if (!std::isfinite(scale)) return QLORA_ERR_INVALID_ARG;
   const qlora_status sh = check_linear_shape(M, K, N, r);
   if (sh != QLORA_OK) return sh;
   if (r % 8 != 0) return QLORA_ERR_UNSUPPORTED;  // no room for the padded adapter here

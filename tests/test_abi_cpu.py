@@ -118,6 +118,53 @@ def test_linear_bwd_validation(L):
     assert L.qlora_linear_bwd(*bad) == 4
 
 
+def fwd_noalloc(L, **kw):
+    a = dict(X=FAKE, M=16, K=256, N=256, codes=FAKE, aq=FAKE, sc=FAKE, A=FAKE, B=FAKE, r=8, s=2.0, Y=FAKE,
+             T=FAKE, st=None)
+    a.update(kw)
+    return L.qlora_linear_fwd_noalloc(a["X"], a["M"], a["K"], a["N"], a["codes"], a["aq"], a["sc"], a["A"], a["B"],
+                                      a["r"], a["s"], a["Y"], a["T"], a["st"])
+
+
+def test_linear_fwd_noalloc_validation(L):
+    """The allocation-free forward takes the same shape rules as the regular
+    one, plus ranks that are multiples of 8 and shapes whose scratch fits its
+    fixed device array (16 MiB)."""
+    assert fwd_noalloc(L, T=None) == 1
+    assert fwd_noalloc(L, s=float("nan")) == 1
+    assert fwd_noalloc(L, s=float("inf")) == 1
+    assert fwd_noalloc(L, s=float("-inf")) == 1
+    assert fwd_noalloc(L, M=0) == 1
+    assert fwd_noalloc(L, K=100) == 3
+    assert fwd_noalloc(L, N=260) == 3
+    assert fwd_noalloc(L, r=257) == 3
+    assert fwd_noalloc(L, r=12) == 3   # not a multiple of 8: no room to pad here
+    assert fwd_noalloc(L, Y=FAKE + 8) == 2
+    assert fwd_noalloc(L, sc=FAKE + 2) == 2
+    assert fwd_noalloc(L, M=65536, K=4096, r=128) == 4  # scratch beyond the fixed array
+
+
+def test_four_bit_entry_points_validate_the_code(L):
+    """The 4-bit calls take NF4, FP4 or Int4, optionally with the centred
+    constants flag; any other code is rejected before the shape checks."""
+    P = FAKE
+    args = [P, 16, 256, 256, P, P, P, None, P, P, 8, 2.0, P, P, P, 1 << 30, None]
+    for code in (3, -1, 0x200, 0x42, 3 | 0x100):  # no such code, stray bits, an unknown flag
+        a = list(args)
+        a[7] = code
+        assert L.qlora_linear_fwd_4bit(*a) == 1, code
+        b = [P, P, P, 16, 256, 256, P, P, P, code, P, P, 8, 2.0, P, P, P, P, 1 << 30, None]
+        assert L.qlora_linear_bwd_4bit(*b) == 1, code
+    for code in (q.qlora.CODES["nf4"], q.qlora.CODES["fp4"], q.qlora.CODES["int4"],
+                 q.qlora.CODES["nf4"] | q.qlora.DQ["centred_fp8"], q.qlora.CODES["int4"] | q.qlora.DQ["centred_fp8"]):
+        a = list(args)
+        a[7] = code
+        a[2] = 100  # valid code: the shape check now decides
+        assert L.qlora_linear_fwd_4bit(*a) == 3, code
+        b = [P, P, P, 16, 100, 256, P, P, P, code, P, P, 8, 2.0, P, P, P, P, 1 << 30, None]
+        assert L.qlora_linear_bwd_4bit(*b) == 3, code
+
+
 def test_codec_validation(L):
     assert L.qlora_quantize_nf4(None, 64, FAKE, FAKE, FAKE, None) == 1
     assert L.qlora_quantize_nf4(FAKE, 0, FAKE, FAKE, FAKE, None) == 1
