@@ -109,10 +109,14 @@ extern "C" {
 void* qlora_paged_malloc(size_t size, int device, void* stream) {
   (void)stream;
   int prev = 0;
-  if (cudaGetDevice(&prev) != cudaSuccess) return nullptr;
-  if (device >= 0 && device != prev && cudaSetDevice(device) != cudaSuccess) return nullptr;
+  cudaError_t e = cudaGetDevice(&prev);
+  if (e == cudaSuccess && device >= 0 && device != prev) e = cudaSetDevice(device);
+  if (e != cudaSuccess) {
+    cuda_fail(e);  // qlora_last_cuda_error says why the result is null
+    return nullptr;
+  }
   void* p = nullptr;
-  const cudaError_t e = cudaMallocManaged(&p, size > 0 ? size : 1, cudaMemAttachGlobal);
+  e = cudaMallocManaged(&p, size > 0 ? size : 1, cudaMemAttachGlobal);
   if (device >= 0 && device != prev) cudaSetDevice(prev);
   if (e != cudaSuccess) {
     cuda_fail(e);

@@ -165,6 +165,16 @@ def test_four_bit_entry_points_validate_the_code(L):
         assert L.qlora_linear_bwd_4bit(*b) == 3, code
 
 
+def test_paged_malloc_without_a_device_reports_why(L):
+    """On a machine without a GPU the unified-memory allocation returns NULL
+    and qlora_last_cuda_error names the CUDA error behind it."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present: the allocation would succeed")
+    assert not L.qlora_paged_malloc(4096, -1, None)
+    assert L.qlora_last_cuda_error()
+
+
 def test_codec_validation(L):
     assert L.qlora_quantize_nf4(None, 64, FAKE, FAKE, FAKE, None) == 1
     assert L.qlora_quantize_nf4(FAKE, 0, FAKE, FAKE, FAKE, None) == 1
