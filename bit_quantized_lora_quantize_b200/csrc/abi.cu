@@ -43,7 +43,7 @@ bool small_m_path(int64_t M, int r) { return M <= kSmallMMax && rank8(r) <= 128;
 // Up to 8 tokens the forward decodes into register fragments of mma.sync
 // (smallm_rd.cu), and up to 16 when the weight has 2^27 elements or more;
 // otherwise, up to 128 tokens, into tensor memory (smallm.cu).  Measured at
-// 16 tokens: 44.0 against 38.9 us for 8192 x 8192, 64.7 against 72.7 us for
+// 16 tokens: 44.0 against 38.9 us for 8192 x 8192, 62.5 against 72.7 us for
 // 22016 x 8192.
 bool small_m_rd_path(int64_t M, int64_t K, int64_t N, int r) {
   if (rank8(r) > 128 || M > kSmallMRdMax) return false;
